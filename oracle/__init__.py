@@ -1,0 +1,141 @@
+"""CPU fp64 oracle for exact scaled-dot-product attention (forward and backward).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may import this package; the product path
+(``io_aware_exact_23_b200``) never does, and the two share no code.
+
+``ref_attn.c`` holds the arithmetic (plain per-row loops in fp64, see its
+header for the passages of the FlashAttention pages it follows);
+``ref_numpy.py`` is an independent whole-matrix NumPy restatement used only
+to cross-check the C code on tiny shapes.  This module compiles the C file
+with gcc on first use and marshals arrays through ctypes.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(closed forms, invariants, finite differences, autograd, hand-derived golden
+fixtures).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ref_attn.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``ref_attn.c`` into ``liboracle.so`` (plain -O2, IEEE fp64)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+             "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        D = ctypes.POINTER(ctypes.c_double)
+        L = ctypes.POINTER(ctypes.c_long)
+        cl, cd, ci = ctypes.c_long, ctypes.c_double, ctypes.c_int
+        lib.ref_attn_fwd.argtypes = [D, D, D, D, D, cl, cl, cl, cl, cd, ci, ci]
+        lib.ref_attn_bwd.argtypes = [D, D, D, D, D, D, D, cl, cl, cl, cl, cd, ci, ci]
+        lib.ref_attn_fwd_rows.argtypes = [D, D, D, cl, cl, cl, cl, cd, ci, L, L, cl, D, D, ci]
+        lib.ref_attn_dq_rows.argtypes = [D, D, D, D, cl, cl, cl, cl, cd, ci, L, L, cl, D, ci]
+        for f in (lib.ref_attn_fwd, lib.ref_attn_bwd, lib.ref_attn_fwd_rows, lib.ref_attn_dq_rows):
+            f.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    """Exact widening of float inputs (bf16/fp32/fp64 tensors or arrays) to fp64."""
+    if hasattr(x, "detach"):  # torch tensor: widen in torch (exact for bf16), then view
+        import torch
+        x = x.detach().to("cpu", torch.float64).contiguous().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _shape4(q):
+    if q.ndim != 4:
+        raise ValueError("expected a [B, H, N, d] tensor")
+    return q.shape
+
+
+def ref_fwd(q, k, v, scale: float, causal: bool, nthreads: int = 0):
+    """O [B,H,N,d] and LSE [B,H,N] in fp64 (vanilla attention, safe softmax)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = _shape4(q)
+    assert k.shape == q.shape and v.shape == q.shape
+    o = np.empty_like(q)
+    lse = np.empty((B, H, N), dtype=np.float64)
+    rc = _load().ref_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                              B, H, N, d, float(scale), int(bool(causal)), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"ref_attn_fwd failed ({rc})")
+    return o, lse
+
+
+def ref_bwd(q, k, v, dO, scale: float, causal: bool, nthreads: int = 0):
+    """dQ, dK, dV [B,H,N,d] in fp64 for the upstream gradient dO."""
+    q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
+    B, H, N, d = _shape4(q)
+    assert k.shape == q.shape and v.shape == q.shape and dO.shape == q.shape
+    dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+    rc = _load().ref_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dq), _ptr(dk), _ptr(dv),
+                              B, H, N, d, float(scale), int(bool(causal)), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"ref_attn_bwd failed ({rc})")
+    return dq, dk, dv
+
+
+def _samples(samp_bh, samp_row):
+    sb = np.ascontiguousarray(np.asarray(samp_bh, dtype=np.int64)).astype(np.dtype("l"))
+    sr = np.ascontiguousarray(np.asarray(samp_row, dtype=np.int64)).astype(np.dtype("l"))
+    assert sb.shape == sr.shape and sb.ndim == 1
+    return sb, sr
+
+
+def ref_fwd_rows(q, k, v, scale: float, causal: bool, samp_bh, samp_row, nthreads: int = 0):
+    """O rows [n, d] and LSE [n] at the sampled (flat head index, query row) pairs."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = _shape4(q)
+    sb, sr = _samples(samp_bh, samp_row)
+    n = sb.shape[0]
+    o = np.empty((n, d), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    Lp = ctypes.POINTER(ctypes.c_long)
+    rc = _load().ref_attn_fwd_rows(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(scale),
+                                   int(bool(causal)), sb.ctypes.data_as(Lp), sr.ctypes.data_as(Lp),
+                                   n, _ptr(o), _ptr(lse), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"ref_attn_fwd_rows failed ({rc})")
+    return o, lse
+
+
+def ref_dq_rows(q, k, v, dO, scale: float, causal: bool, samp_bh, samp_row, nthreads: int = 0):
+    """dQ rows [n, d] at the sampled (flat head index, query row) pairs."""
+    q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
+    B, H, N, d = _shape4(q)
+    sb, sr = _samples(samp_bh, samp_row)
+    n = sb.shape[0]
+    dq = np.empty((n, d), dtype=np.float64)
+    Lp = ctypes.POINTER(ctypes.c_long)
+    rc = _load().ref_attn_dq_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), B, H, N, d, float(scale),
+                                  int(bool(causal)), sb.ctypes.data_as(Lp), sr.ctypes.data_as(Lp),
+                                  n, _ptr(dq), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"ref_attn_dq_rows failed ({rc})")
+    return dq
