@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Throughput of one fused attention training step (forward + backward) on B200.
+
+A step is one pass of the whole hot path over one batch: ``fa_fwd`` (O, LSE)
+then ``fa_bwd`` (D preprocess, dK/dV/dQ kernel, dQ conversion) on the
+workload B=2, H=32, N=4096, d=128, causal -- the first configuration at the
+N >= 4096, d = 128 point where the throughput targets are stated.  Inputs are
+synthetic (seeded N(0,1) rounded to bf16) and already resident in HBM when the
+timed region starts; Q, K, V and dO alone are 268 MB, larger than the 126 MB L2,
+so no L2 flush is inserted between steps.
+
+Counted FLOPs: forward 4*B*H*N^2*d, backward 2.5x that, both halved for causal.
+
+Launch: ``python bench.py --gpus N --steps K --warmup W`` (one rank per GPU
+under torchrun for N > 1; every rank runs the same workload: weak scaling, no
+data-path collective).  Prints one JSON line on rank 0.
+``--impl reference`` times the CPU fp64 oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd and fwd+bwd TFLOP/s (bf16, 1×B200) and % of tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["io_aware_exact_23_b200/csrc/ptx.cuh", "io_aware_exact_23_b200/csrc/fa_fwd.cuh",
+                  "io_aware_exact_23_b200/csrc/fa_bwd.cuh", "io_aware_exact_23_b200/csrc/fa_api.cu"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="b2h32n4096d128_causal")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0,
+                    help="seconds of oracle work for the cpu_baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu capture, if the kernels have not changed since."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    for r in rec.get("records", []):
+        if r.get("kernel") == kernel and r.get("workload") == workload and r.get("source_sha") == source_sha():
+            return r.get("dram_bytes_per_launch")
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling; keeps samples taken inside [t0, t1]."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.samples = []
+        self.proc = None
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
+        if gpu_id:
+            cmd[1:1] = ["-i", gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.samples:
+            if not (t0 <= ts <= t1):
+                continue
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def rank_workload(w, rank: int):
+    """Rank r's shard of the global batch: the same shape, its own seed (r)."""
+    import dataclasses
+    return dataclasses.replace(w, seed=w.seed + rank)
+
+
+def reduce_max(values, dist, device):
+    """Element-wise max over ranks (device timing: the slowest rank sets the time)."""
+    import torch
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def cpu_baseline_sample(w, budget_s: float):
+    """Time the oracle (as it stands) on whole heads of the workload until the budget is spent."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from io_aware_exact_23_b200.inputs import make_inputs
+    t = make_inputs(w)  # CPU tensors
+    cores = os.cpu_count() or 1
+    oracle.build()
+    heads, flops, secs = 0, 0.0, 0.0
+    per_head = (w.fwd_flops() + w.bwd_flops()) / (w.B * w.H)
+    for bh in range(w.B * w.H):
+        b, h = divmod(bh, w.H)
+        sl = {k: v[b:b + 1, h:h + 1] for k, v in t.items()}
+        t0 = time.perf_counter()
+        oracle.ref_fwd(sl["q"], sl["k"], sl["v"], w.scale, w.causal, nthreads=cores)
+        oracle.ref_bwd(sl["q"], sl["k"], sl["v"], sl["do"], w.scale, w.causal, nthreads=cores)
+        secs += time.perf_counter() - t0
+        heads += 1
+        flops += per_head
+        if secs >= budget_s:
+            break
+    del np, torch
+    return {"value": flops / secs / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{heads} of {w.B * w.H} heads (b,h in order) of {w.name}, forward + backward, "
+                      f"fp64 C oracle with {cores} threads, {secs:.1f} s"}
+
+
+def run_reference(args, w, world, rank):
+    """--impl reference: the CPU oracle on the same workload, one head per step (rank 0 only)."""
+    if rank != 0:
+        return 0
+    import oracle
+    from io_aware_exact_23_b200.inputs import make_inputs
+    cores = os.cpu_count() or 1
+    oracle.build()
+    t = make_inputs(w)
+    per_head = (w.fwd_flops() + w.bwd_flops()) / (w.B * w.H)
+    BH = w.B * w.H
+
+    def step(s):
+        b, h = divmod(s % BH, w.H)
+        sl = {k: v[b:b + 1, h:h + 1] for k, v in t.items()}
+        oracle.ref_fwd(sl["q"], sl["k"], sl["v"], w.scale, w.causal, nthreads=cores)
+        oracle.ref_bwd(sl["q"], sl["k"], sl["v"], sl["do"], w.scale, w.causal, nthreads=cores)
+
+    for s in range(args.warmup):
+        step(s)
+    t0 = time.perf_counter()
+    done = 0
+    for s in range(args.steps):
+        step(args.warmup + s)
+        done += 1
+        if time.perf_counter() - t0 > 240.0:  # keep the arm within a few minutes
+            break
+    secs = time.perf_counter() - t0
+    value = per_head * done / secs / 1e12
+    sample = (f"one (b,h) head of {w.name} per step (fwd + bwd, fp64 C oracle, {cores} threads), "
+              f"{done} steps")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": world,
+            "steps": done, "warmup": args.warmup, "ms_per_step": secs / done * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                       "step": "one head of the workload (CPU oracle)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup()
+    from io_aware_exact_23_b200.inputs import CONFIGS
+    w = CONFIGS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w, world, rank)
+
+    import torch
+    import torch.distributed as dist
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the attention path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    from io_aware_exact_23_b200 import binding as fa
+    from io_aware_exact_23_b200.inputs import make_inputs, score_matrix_bytes
+
+    dev = torch.device("cuda", local)
+    t = make_inputs(rank_workload(w, rank), device=dev)
+    q, k, v, dO = t["q"], t["k"], t["v"], t["do"]
+    B, H, N, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws = torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats(dev)
+
+    def step(ev_f=None, ev_b=None):
+        if ev_f is not None:
+            ev_f[0].record()
+        fa.fa_fwd(q, k, v, o, lse, w.scale, w.causal)
+        if ev_f is not None:
+            ev_f[1].record()
+        fa.fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, w.scale, w.causal, ws, events=ev_b)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    if fa.fa_device_status() != 0:
+        raise SystemExit("bench.py: device status error during warm-up")
+
+    K = args.steps
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    ev_f = [(mk(), mk()) for _ in range(K)]
+    ev_b = [tuple(mk() for _ in range(4)) for _ in range(K)]
+    start, end = mk(), mk()
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    tw0 = time.time()
+    start.record()
+    for s in range(K):
+        step(ev_f[s], ev_b[s])
+    end.record()
+    torch.cuda.synchronize()
+    tw1 = time.time()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    status = fa.fa_device_status()
+    ms = start.elapsed_time(end)
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_f)
+    pre_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev_b)
+    main_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev_b)
+    conv_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev_b)
+    bwd_ms = statistics.mean(e[0].elapsed_time(e[3]) for e in ev_b)
+    peak_mem = torch.cuda.max_memory_allocated(dev)  # inputs + outputs + workspace
+    ms, fwd_ms, bwd_ms, main_ms, pre_ms, conv_ms, status = reduce_max(
+        [ms, fwd_ms, bwd_ms, main_ms, pre_ms, conv_ms, float(status)], dist, dev)
+
+    # ---------------------------------------------------------------- e2e
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = {nm: t[nm].cpu().pin_memory() for nm in ("q", "k", "v", "do")}
+        out_h = {"o": torch.empty(o.shape, dtype=o.dtype, pin_memory=True),
+                 "lse": torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True),
+                 "dq": torch.empty(dq.shape, dtype=dq.dtype, pin_memory=True),
+                 "dk": torch.empty(dk.shape, dtype=dk.dtype, pin_memory=True),
+                 "dv": torch.empty(dv.shape, dtype=dv.dtype, pin_memory=True)}
+        h2d = sum(x.numel() * x.element_size() for x in pin.values())
+        d2h = sum(x.numel() * x.element_size() for x in out_h.values())
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = mk(), mk()
+        e0.record()
+        for _ in range(args.e2e_steps):
+            q.copy_(pin["q"], non_blocking=True)
+            k.copy_(pin["k"], non_blocking=True)
+            v.copy_(pin["v"], non_blocking=True)
+            dO.copy_(pin["do"], non_blocking=True)
+            step()
+            out_h["o"].copy_(o, non_blocking=True)
+            out_h["lse"].copy_(lse, non_blocking=True)
+            out_h["dq"].copy_(dq, non_blocking=True)
+            out_h["dk"].copy_(dk, non_blocking=True)
+            out_h["dv"].copy_(dv, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = reduce_max([e0.elapsed_time(e1) / args.e2e_steps], dist, dev)[0]
+        e2e = {"value": world * (w.fwd_flops() + w.bwd_flops()) / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "path": "pinned host -> device copies, fa_fwd + fa_bwd through the C ABI, outputs -> pinned host"}
+
+    if rank == 0:
+        peaks, peak_kind = load_peaks()
+        flops_step = w.fwd_flops() + w.bwd_flops()
+        value = world * flops_step * K / (ms / 1e3) / 1e12
+        fwd_tf = w.fwd_flops() / (fwd_ms / 1e3) / 1e12
+        bwd_tf = w.bwd_flops() / (bwd_ms / 1e3) / 1e12
+        main_tf = w.bwd_flops() / (main_ms / 1e3) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        peak_sus = float(peaks.get("bf16_tflops_sustained", peak))
+        kernels = {"fa_fwd_kernel": fwd_ms, "fa_bwd_pre_kernel": pre_ms, "fa_bwd_kernel": main_ms,
+                   "fa_dq_convert_kernel": conv_ms}
+        dominant = max(kernels, key=kernels.get)
+        dom_flops = w.bwd_flops() if dominant in ("fa_bwd_kernel",) else (
+            w.fwd_flops() if dominant == "fa_fwd_kernel" else 0.0)
+        dom_tf = dom_flops / (kernels[dominant] / 1e3) / 1e12
+        clocks = sampler.summary(tw0, tw1)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
+                       "per_rank": "the full workload on every rank (independent heads, no collective)",
+                       "l2": "no flush: Q, K, V, dO total 268 MB, larger than the 126 MB L2"},
+            "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+            "fwd_frac_of_peak": fwd_tf / peak, "bwd_frac_of_peak": bwd_tf / peak,
+            "kernel_ms": kernels,
+            "roofline": {"bound": "tensor", "kernel": dominant, "achieved": dom_tf, "peak": peak,
+                         "unit": "TFLOP/s", "frac": dom_tf / peak,
+                         "peak_kind": f"bf16 dense, burst, {peak_kind} (MEASURED_PEAKS.json)",
+                         "frac_of_sustained": dom_tf / peak_sus,
+                         "traffic": stored_traffic(dominant, w.name)},
+            "peak_hbm_bytes": peak_mem,
+            "score_matrix_bytes_bf16": score_matrix_bytes(B, H, N, 2),
+            "clocks": clocks,
+            "gpu_launches": 4 * K,
+            "device_status": int(status),
+        }
+        if e2e is not None:
+            line["e2e"] = e2e
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline_sample(w, args.cpu_budget_s)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,136 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact scaled-dot-product attention, forward and
+ * backward, as fused tiled kernels for NVIDIA B200 (sm_100a).
+ *
+ * What is computed (per head (b, h); heads are independent):
+ *
+ *   O = softmax(scale * Q K^T [+ causal mask]) V
+ *
+ * -- the "Vanilla Attention" definition of the FlashAttention review
+ * (mrodiduger, "Vanilla Attention", with the scale the review leaves out),
+ * computed the IO-aware way the same review ("Tiling", "Recomputation") and the
+ * FlashAttention summary ("Architecture, step by step") describe: tiles of
+ * Q, K and V are staged on chip, a running max m and normaliser l combine the
+ * blocks (online softmax), and only O and the per-row statistics reach HBM.
+ * The N x N score matrix is never written to memory.  The statistics are
+ * stored folded into one log-sum-exp, LSE_i = m_i + ln(l_i) (natural log).
+ * The backward pass recomputes S and P from Q, K and LSE
+ * ("Recomputation") and returns dQ, dK, dV for an upstream gradient dO.
+ *
+ * Causal mask: key j is masked (-inf) for query i when j > i (the diagonal is
+ * kept; queries and keys share positions 0..N-1).
+ *
+ * Layout and types (all tensors caller-owned, device memory, contiguous):
+ *   q, k, v, o, dO, dq, dk, dv : [B, H, N, d] bf16 (passed as raw 16-bit words)
+ *   lse                        : [B, H, N] fp32, natural-log LSE
+ *   workspace (fa_bwd only)    : fa_bwd_workspace_bytes(B, H, N, d) bytes
+ * Every pointer must be 16-byte aligned (a TMA requirement).  Outputs must not
+ * overlap inputs.  Inputs are never written.
+ *
+ * Supported: d in {64, 128}; B, H, N >= 1; B*H*N*d < 2^31 elements per tensor;
+ * scale finite and > 0; causal in {0, 1}; an sm_100 device.
+ *
+ * Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ * default stream).  The return value reports argument and launch errors only;
+ * on an argument error nothing is launched and no output is touched.  A
+ * device-side failure (a pipeline wait that exceeded its time limit) is
+ * recorded in a library-owned device status word and returned by
+ * fa_device_status().  No exception crosses this interface.  The library
+ * allocates only that status word (32 bytes per device, once, on the first
+ * call that reaches the device) and host-side state; all tensors and the
+ * workspace come from the caller.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,   /* null pointer, N/B/H < 1, bad scale or causal flag */
+    FA_ERR_UNSUPPORTED = 2,   /* d not in {64,128}, tensor too large, device not sm_100 */
+    FA_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned */
+    FA_ERR_WORKSPACE = 4,     /* workspace null or smaller than fa_bwd_workspace_bytes() */
+    FA_ERR_NO_DEVICE = 5,     /* no CUDA device could be used */
+    FA_ERR_CUDA = 6,          /* a CUDA runtime/driver call or a launch failed */
+    FA_ERR_DEVICE_TIMEOUT = 7, /* a kernel gave up on a pipeline wait (fa_device_status) */
+    FA_ERR_DEVICE_INTERNAL = 8 /* a kernel found its launch environment unusable
+                                  (e.g. a misaligned shared-memory window) */
+} fa_status;
+
+/*
+ * Forward pass.  Writes o [B,H,N,d] bf16 and lse [B,H,N] fp32.
+ * Source: FlashAttention summary "Architecture, step by step" (tile inputs,
+ * compute locally, online normalisation, write compact output) and the review's
+ * "Tiling" section (online softmax instead of the three-loop safe softmax).
+ */
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+           int B, int H, int N, int d, float scale, int causal, void *stream);
+
+/*
+ * Bytes of scratch fa_bwd needs: an fp32 dQ accumulator [B,H,N,d], plus two
+ * fp32 vectors [B,H,Np] with Np = N rounded up to a multiple of 128 -- the
+ * per-row D_i = rowsum(dO * O) and LSE_i * log2(e) -- so
+ * 4*B*H*(N*d + 2*Np) bytes, rounded up to a multiple of 256.
+ * Returns 0 for unsupported or invalid shapes.
+ */
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Backward pass.  Given the forward inputs, its outputs o and lse, and the
+ * upstream gradient dO, writes dq, dk, dv [B,H,N,d] bf16.  Source: the review's
+ * "Recomputation" section (keep the softmax statistics, recompute S and P in the
+ * backward pass); the gradient formulas are the chain rule through softmax.
+ * `workspace` (device, 16-byte aligned, caller-owned, contents ignored on entry)
+ * must hold fa_bwd_workspace_bytes(B,H,N,d) bytes; it is overwritten.
+ */
+int fa_bwd(const void *q, const void *k, const void *v, const void *o,
+           const void *dO, const float *lse, void *dq, void *dk, void *dv,
+           int B, int H, int N, int d, float scale, int causal,
+           void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * fa_bwd with stage timing.  `events` is either NULL (then this is exactly
+ * fa_bwd) or a host array of four cudaEvent_t handles owned by the caller;
+ * they are recorded on `stream` before the preprocess kernel, after it, after
+ * the main dK/dV/dQ kernel, and after the dQ conversion, so the caller can time
+ * each kernel with cudaEventElapsedTime.  Same arguments, layout and errors as
+ * fa_bwd; FA_ERR_CUDA if recording an event fails.
+ */
+int fa_bwd_profiled(const void *q, const void *k, const void *v, const void *o,
+                    const void *dO, const float *lse, void *dq, void *dk,
+                    void *dv, int B, int H, int N, int d, float scale,
+                    int causal, void *workspace, size_t workspace_bytes,
+                    void *stream, void *const *events);
+
+/* Static, human-readable name of a status code (never NULL). */
+const char *fa_status_string(int status);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word of the
+ * current device: FA_OK, or FA_ERR_DEVICE_TIMEOUT if a kernel launched since
+ * the last call gave up on a wait (its outputs are then undefined).
+ * Returns FA_ERR_CUDA if the synchronisation itself fails.
+ */
+int fa_device_status(void *stream);
+
+/*
+ * Like fa_device_status(), and also copies the failure record into info[0..3]:
+ * {kernel id (1 fwd, 2 bwd, 3 bwd preprocess, 4 dQ convert), wait tag, block
+ * index, launch sequence number}; zeros when there was no failure.  `info` is a
+ * host pointer to 4 ints (may be NULL).
+ */
+int fa_device_status_info(void *stream, int *info);
+
+/* Library version, MAJOR*10000 + MINOR*100 + PATCH. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -1,0 +1,155 @@
+"""ctypes binding of libfa.so: argument marshalling only.
+
+Every function here checks tensor dtypes/shapes/devices, turns torch tensors
+into raw device pointers and the current CUDA stream into a handle, and calls
+the C entry point of the same name declared in ``include/fa.h``.  All
+arithmetic happens in the CUDA kernels.  If ``libfa.so`` is missing this module
+raises at import: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
+
+FA_OK = 0
+STATUS_NAMES = {
+    0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_MISALIGNED",
+    4: "FA_ERR_WORKSPACE", 5: "FA_ERR_NO_DEVICE", 6: "FA_ERR_CUDA", 7: "FA_ERR_DEVICE_TIMEOUT",
+    8: "FA_ERR_DEVICE_INTERNAL",
+}
+
+
+class FaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {lib().fa_status_string(code).decode()} ({code})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libfa.so (raises ImportError if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(
+                f"{_LIB_PATH} not found: build it with `python -m io_aware_exact_23_b200.build` "
+                "(the attention path has no CPU fallback)")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+        L.fa_fwd.restype = i
+        L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
+        L.fa_bwd.restype = i
+        L.fa_bwd_profiled.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp,
+                                      ctypes.POINTER(vp)]
+        L.fa_bwd_profiled.restype = i
+        L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
+        L.fa_bwd_workspace_bytes.restype = sz
+        L.fa_status_string.argtypes = [i]
+        L.fa_status_string.restype = ctypes.c_char_p
+        L.fa_device_status.argtypes = [vp]
+        L.fa_device_status.restype = i
+        L.fa_device_status_info.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+        L.fa_device_status_info.restype = i
+        L.fa_version.argtypes = []
+        L.fa_version.restype = i
+        _lib = L
+    return _lib
+
+
+lib()  # fail at import when the extension is missing
+
+
+def _stream_handle(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _check(t: torch.Tensor, name: str, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def fa_fwd(q, k, v, o, lse, scale: float, causal: bool, stream=None) -> None:
+    """O and LSE into the preallocated ``o`` [B,H,N,d] bf16 and ``lse`` [B,H,N] fp32."""
+    B, H, N, d = q.shape
+    for nm, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _check(t, nm, torch.bfloat16, (B, H, N, d))
+    _check(lse, "lse", torch.float32, (B, H, N))
+    rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                      B, H, N, d, float(scale), int(bool(causal)), _stream_handle(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd")
+
+
+def fa_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().fa_bwd_workspace_bytes(B, H, N, d))
+
+
+def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, scale: float, causal: bool, workspace, stream=None,
+           events=None) -> None:
+    """dQ, dK, dV into preallocated bf16 tensors; ``workspace`` is a uint8 CUDA tensor.
+
+    ``events``: optional sequence of four ``torch.cuda.Event(enable_timing=True)``
+    recorded around the preprocess, main and dQ-conversion kernels.
+    """
+    B, H, N, d = q.shape
+    for nm, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dO", dO), ("dq", dq), ("dk", dk), ("dv", dv)):
+        _check(t, nm, torch.bfloat16, (B, H, N, d))
+    _check(lse, "lse", torch.float32, (B, H, N))
+    _check(workspace, "workspace", torch.uint8)
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dO.data_ptr(), lse.data_ptr(),
+            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, float(scale), int(bool(causal)),
+            workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+    if events is None:
+        rc = lib().fa_bwd(*args)
+    else:
+        if len(events) != 4:
+            raise ValueError("events must hold four torch.cuda.Event objects")
+        handles = (ctypes.c_void_p * 4)(*[ev.cuda_event for ev in events])
+        rc = lib().fa_bwd_profiled(*args, handles)
+    if rc != FA_OK:
+        raise FaError(rc, "fa_bwd")
+
+
+def fa_device_status(stream=None, info: bool = False):
+    """Synchronise the stream and return (and clear) the device status code."""
+    buf = (ctypes.c_int * 4)()
+    rc = lib().fa_device_status_info(_stream_handle(stream), buf)
+    return (rc, list(buf)) if info else rc
+
+
+class Attention:
+    """Allocating convenience wrapper: ``forward`` and ``backward`` on torch tensors."""
+
+    def __init__(self, scale: float, causal: bool):
+        self.scale = float(scale)
+        self.causal = bool(causal)
+
+    def forward(self, q, k, v):
+        B, H, N, d = q.shape
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+        fa_fwd(q, k, v, o, lse, self.scale, self.causal)
+        return o, lse
+
+    def backward(self, q, k, v, o, lse, dO):
+        B, H, N, d = q.shape
+        ws = torch.empty(fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=q.device)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, self.scale, self.causal, ws)
+        return dq, dk, dv

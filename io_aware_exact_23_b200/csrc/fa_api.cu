@@ -1,0 +1,294 @@
+// fa_api.cu -- the C ABI of libfa.so (declared in include/fa.h): argument
+// validation, TMA descriptor encoding, the per-device status block, and the
+// launches of the forward and backward kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kStatusInts = 8;
+
+struct DeviceState {
+  bool ready = false;
+  int *status = nullptr;  // kStatusInts ints, device memory
+  int num_sms = 0;
+  bool attrs_set = false;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+std::atomic<int> g_seq{1};
+
+int next_seq() {
+  int s = g_seq.fetch_add(1);
+  if (s <= 0) {  // wrapped: sequence numbers stay positive (0 marks "none")
+    g_seq.store(2);
+    s = 1;
+  }
+  return s;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [BH, N, D] tensor viewed as 3-D (x = feature, y = row, z = head); box of
+// 64 (or 32 for fp32) features x 128 rows x 1 head, 128-byte swizzle, zero fill.
+int encode_3d(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int elem_bytes, int D, int N, int BH,
+              int box_x) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return FA_ERR_CUDA;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * elem_bytes,
+                           static_cast<cuuint64_t>(N) * D * elem_bytes};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_x), 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(m, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+int encode_bf16(CUtensorMap *m, const void *ptr, int D, int N, int BH) {
+  return encode_3d(m, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH, 64);
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks shared by both passes (no CUDA calls).
+int check_shape(int B, int H, int N, int d, float scale, int causal) {
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long double elems = static_cast<long double>(B) * H * N * d;
+  if (elems >= 2147483648.0L) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+// Lazily set up the current device: compute capability check, SM count and
+// the status block.  Returns a status code.
+int device_state(DeviceState **out, int *dev_out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    cudaGetLastError();
+    return FA_ERR_NO_DEVICE;
+  }
+  if (dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState &s = g_dev[dev];
+  if (!s.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_NO_DEVICE;
+    }
+    if (major != 10 || minor != 0) return FA_ERR_UNSUPPORTED;
+    int *st = nullptr;
+    if (cudaMalloc(&st, kStatusInts * sizeof(int)) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    if (cudaMemset(st, 0, kStatusInts * sizeof(int)) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(st);
+      return FA_ERR_CUDA;
+    }
+    s.status = st;
+    s.num_sms = sms;
+    s.ready = true;
+  }
+  if (!s.attrs_set) {
+    cudaError_t e = cudaSuccess;
+    e = (e == cudaSuccess) ? cudaFuncSetAttribute(fa::fa_fwd_kernel<64, false>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  fa::FwdCfg<64>::kSmemBytes)
+                           : e;
+    e = (e == cudaSuccess) ? cudaFuncSetAttribute(fa::fa_fwd_kernel<64, true>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  fa::FwdCfg<64>::kSmemBytes)
+                           : e;
+    e = (e == cudaSuccess) ? cudaFuncSetAttribute(fa::fa_fwd_kernel<128, false>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  fa::FwdCfg<128>::kSmemBytes)
+                           : e;
+    e = (e == cudaSuccess) ? cudaFuncSetAttribute(fa::fa_fwd_kernel<128, true>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  fa::FwdCfg<128>::kSmemBytes)
+                           : e;
+    e = (e == cudaSuccess) ? fa::bwd_set_attributes() : e;
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    s.attrs_set = true;
+  }
+  *out = &s;
+  if (dev_out) *dev_out = dev;
+  return FA_OK;
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch_fwd(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v, const CUtensorMap &o,
+                       const fa::FwdParams &p, cudaStream_t stream) {
+  const dim3 grid(static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.n_qpairs));
+  fa::fa_fwd_kernel<D, CAUSAL><<<grid, fa::FwdCfg<D>::kThreads, fa::FwdCfg<D>::kSmemBytes, stream>>>(q, k, v, o, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return 100; }
+
+const char *fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: invalid argument";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: unsupported shape or device";
+    case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED: pointer not 16-byte aligned";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace missing or too small";
+    case FA_ERR_NO_DEVICE: return "FA_ERR_NO_DEVICE: no usable CUDA device";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA call or launch failed";
+    case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT: a kernel gave up on a pipeline wait";
+    case FA_ERR_DEVICE_INTERNAL: return "FA_ERR_DEVICE_INTERNAL: kernel launch environment unusable";
+    default: return "unknown fa_status";
+  }
+}
+
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N, int d,
+           float scale, int causal, void *stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  int st = check_shape(B, H, N, d, scale, causal);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+  DeviceState *ds = nullptr;
+  st = device_state(&ds, nullptr);
+  if (st != FA_OK) return st;
+
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv, to;
+  if (encode_bf16(&tq, q, d, N, BH) || encode_bf16(&tk, k, d, N, BH) || encode_bf16(&tv, v, d, N, BH) ||
+      encode_bf16(&to, o, d, N, BH))
+    return FA_ERR_CUDA;
+  fa::FwdParams p;
+  p.lse = lse;
+  p.status = ds->status;
+  p.seq = next_seq();
+  p.N = N;
+  p.BH = BH;
+  p.n_qpairs = (N + 255) / 256;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (d == 64)
+    e = causal ? launch_fwd<64, true>(tq, tk, tv, to, p, s) : launch_fwd<64, false>(tq, tk, tv, to, p, s);
+  else
+    e = causal ? launch_fwd<128, true>(tq, tk, tv, to, p, s) : launch_fwd<128, false>(tq, tk, tv, to, p, s);
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (check_shape(B, H, N, d, 1.f, 0) != FA_OK) return 0;
+  return fa::bwd_workspace_bytes(B * H, N, d);
+}
+
+int fa_bwd_profiled(const void *q, const void *k, const void *v, const void *o, const void *dO,
+                    const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale,
+                    int causal, void *workspace, size_t workspace_bytes, void *stream, void *const *events) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  int st = check_shape(B, H, N, d, scale, causal);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_MISALIGNED;
+  const int BH = B * H;
+  if (!workspace || workspace_bytes < fa::bwd_workspace_bytes(BH, N, d)) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+  if (events && (!events[0] || !events[1] || !events[2] || !events[3])) return FA_ERR_INVALID_ARG;
+  DeviceState *ds = nullptr;
+  st = device_state(&ds, nullptr);
+  if (st != FA_OK) return st;
+
+  fa::BwdLaunch L;
+  L.q = q; L.k = k; L.v = v; L.o = o; L.dO = dO; L.lse = lse;
+  L.dq = dq; L.dk = dk; L.dv = dv;
+  L.BH = BH; L.N = N; L.d = d; L.scale = scale; L.causal = causal;
+  L.workspace = workspace;
+  L.status = ds->status;
+  L.seq = next_seq();
+  L.num_sms = ds->num_sms;
+  L.events = reinterpret_cast<cudaEvent_t const *>(events);
+  CUtensorMap maps[6];
+  if (encode_bf16(&maps[0], q, d, N, BH) || encode_bf16(&maps[1], k, d, N, BH) ||
+      encode_bf16(&maps[2], v, d, N, BH) || encode_bf16(&maps[3], dO, d, N, BH) ||
+      encode_bf16(&maps[4], dk, d, N, BH) || encode_bf16(&maps[5], dv, d, N, BH))
+    return FA_ERR_CUDA;
+  cudaError_t e = fa::bwd_launch(L, maps, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dO, const float *lse, void *dq,
+           void *dk, void *dv, int B, int H, int N, int d, float scale, int causal, void *workspace,
+           size_t workspace_bytes, void *stream) {
+  return fa_bwd_profiled(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes,
+                         stream, nullptr);
+}
+
+int fa_device_status_info(void *stream, int *info) {
+  if (info) std::memset(info, 0, 4 * sizeof(int));
+  DeviceState *ds = nullptr;
+  int st = device_state(&ds, nullptr);
+  if (st != FA_OK) return st;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  int h[kStatusInts];
+  if (cudaMemcpy(h, ds->status, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  if (h[0] == 0) return FA_OK;
+  if (info) {
+    info[0] = h[1];
+    info[1] = h[2];
+    info[2] = h[3];
+    info[3] = h[4];
+  }
+  if (cudaMemset(ds->status, 0, kStatusInts * sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  return h[0] == fa::kStatusInternal ? FA_ERR_DEVICE_INTERNAL : FA_ERR_DEVICE_TIMEOUT;
+}
+
+int fa_device_status(void *stream) { return fa_device_status_info(stream, nullptr); }
+
+}  // extern "C"

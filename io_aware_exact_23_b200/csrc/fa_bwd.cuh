@@ -1,0 +1,561 @@
+// fa_bwd.cuh -- exact-attention backward pass for sm_100a.
+//
+// The backward pass keeps no N x N matrix either: following the review's
+// "Recomputation" section, it rebuilds S and P tile by tile from Q, K and the
+// stored log-sum-exp, P_ij = 2^(c*S_ij - LSE_i*log2(e)).  The gradients are the
+// chain rule through softmax:
+//   dV = P^T dO,  dP = dO V^T,  dS = P o (dP - D),  D_i = sum_k dO_ik O_ik,
+//   dQ = scale * dS K,  dK = scale * dS^T Q.
+//
+// Three kernels on one stream:
+//   1. fa_bwd_pre_kernel   D_i = rowsum(dO o O) and LSE_i*log2(e) into the
+//                          workspace (padded to whole 128-row tiles), and zero
+//                          the fp32 dQ accumulator.
+//   2. fa_bwd_kernel       one CTA per (head, 128-row key tile j): K_j, V_j stay
+//                          in smem, dK_j and dV_j accumulate in TMEM while the
+//                          CTA walks the query tiles; each query tile's dQ
+//                          contribution is added into the fp32 accumulator.
+//   3. fa_dq_convert_kernel  dQ (bf16) = accumulator.
+//
+// fa_bwd_kernel roles (448 threads):
+//   warps 0-3   compute, query columns 0..63 of each tile (thread = key row)
+//   warps 4-7   compute, query columns 64..127
+//   warps 8-11  dQ drain: TMEM dQ rows -> fp32 adds into the accumulator
+//   warp  12    TMA producer: K_j, V_j once; Q_i, dO_i, LSE_i, D_i per tile (2 stages)
+//   warp  13    MMA issuer (one thread), five MMAs per query tile:
+//                 S^T  = K_j Q_i^T      (smem x smem)      -> TMEM
+//                 dP^T = V_j dO_i^T     (smem x smem)      -> TMEM
+//                 dV  += P^T dO_i       (TMEM x smem)
+//                 dK  += dS^T Q_i       (smem x smem)
+//                 dQ_i = dS K_j         (smem x smem, dS read transposed)
+//
+// TMEM columns (512): S^T [0,128) with P^T (bf16) over its first 64 columns;
+// dP^T [128,256); dK [256,256+D); dV [256+D,256+2D); dQ reuses dP^T's columns
+// when D = 128 (dP^T is dead once dS is formed) and [384,448) when D = 64.
+// dS^T (bf16) is written to smem in the 128-byte-swizzled K-major layout,
+// which is at the same time the MN-major layout of dS for the dQ MMA.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace fa {
+
+struct BwdParams {
+  const float *ws_lse2;  // [BH, Npad]  LSE * log2(e), +inf on padded rows
+  const float *ws_D;     // [BH, Npad]  rowsum(dO o O), 0 on padded rows
+  float *ws_dq;          // [BH, N, D]  fp32 dQ accumulator (zeroed by the preprocess)
+  int *status;
+  int seq;
+  int N;
+  int Npad;
+  int BH;
+  float scale_log2;
+  float scale;
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kTile = 128 * D * 2;
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kTile;
+  static constexpr int kOffQ = 2 * kTile;   // [2]
+  static constexpr int kOffdO = 4 * kTile;  // [2]
+  static constexpr int kOffdS = 6 * kTile;  // 128 x 128 bf16
+  static constexpr int kOffL = kOffdS + 32768;  // [2][128] fp32
+  static constexpr int kOffDv = kOffL + 1024;   // [2][128] fp32
+  static constexpr int kOffBar = kOffDv + 1024;
+  static constexpr int kSmemBytes = kOffBar + 256;
+  static constexpr int kThreads = 448;
+  static constexpr uint32_t kColS = 0, kColdP = 128, kColdK = 256, kColdV = 256 + D;
+  static constexpr uint32_t kColdQ = (D == 128) ? 128 : 384;
+};
+
+enum BwdTag : int {
+  kBTagKV = 11, kBTagQdoFull = 12, kBTagQdoEmpty = 13, kBTagSFull = 14, kBTagDpFull = 15, kBTagPFull = 16,
+  kBTagDsFull = 17, kBTagDvDone = 18, kBTagDkqDone = 19, kBTagDqEmpty = 20, kBTagEpi = 21
+};
+
+__device__ __forceinline__ uint32_t bsw128(int row, int chunk) {
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+// ----------------------------------------------------------- preprocess
+// Lanes-per-row = D / 8 (each lane handles 8 features = 16 bytes).
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t *__restrict__ o,
+                                                         const uint16_t *__restrict__ dO,
+                                                         const float *__restrict__ lse, float *__restrict__ ws_D,
+                                                         float *__restrict__ ws_lse2, float *__restrict__ ws_dq,
+                                                         int N, int Npad, int BH) {
+  constexpr int LPR = D / 8;
+  constexpr int RPW = 32 / LPR;  // rows per warp pass
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / LPR, part = lane % LPR;
+  const long warps = static_cast<long>(gridDim.x) * (blockDim.x / 32);
+  const long gw = static_cast<long>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const long rows = static_cast<long>(BH) * Npad;
+  for (long base = gw * RPW; base < rows; base += warps * RPW) {
+    const long row = base + sub;
+    float acc = 0.f;
+    const bool in = row < rows;
+    const int bh = in ? static_cast<int>(row / Npad) : 0;
+    const int i = in ? static_cast<int>(row % Npad) : 0;
+    const bool valid = in && i < N;
+    if (valid) {
+      const size_t off = (static_cast<size_t>(bh) * N + i) * D + part * 8;
+      const uint4 a = *reinterpret_cast<const uint4 *>(o + off);
+      const uint4 b = *reinterpret_cast<const uint4 *>(dO + off);
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        acc = fmaf(__uint_as_float(av[t] << 16), __uint_as_float(bv[t] << 16), acc);
+        acc = fmaf(__uint_as_float(av[t] & 0xFFFF0000u), __uint_as_float(bv[t] & 0xFFFF0000u), acc);
+      }
+    }
+#pragma unroll
+    for (int w = LPR / 2; w >= 1; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
+    if (in && part == 0) {
+      ws_D[row] = valid ? acc : 0.f;
+      ws_lse2[row] = valid ? lse[static_cast<size_t>(bh) * N + i] * 1.4426950408889634f : INFINITY;
+    }
+  }
+  const long n4 = static_cast<long>(BH) * N * D / 4;
+  const long tid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long nthreads = static_cast<long>(gridDim.x) * blockDim.x;
+  float4 *z = reinterpret_cast<float4 *>(ws_dq);
+  for (long t = tid; t < n4; t += nthreads) z[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// --------------------------------------------------------- dQ conversion
+__global__ void __launch_bounds__(256) fa_dq_convert_kernel(const float *__restrict__ ws_dq,
+                                                            uint16_t *__restrict__ dq, long n4) {
+  const long tid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long nthreads = static_cast<long>(gridDim.x) * blockDim.x;
+  const float4 *src = reinterpret_cast<const float4 *>(ws_dq);
+  uint2 *dst = reinterpret_cast<uint2 *>(dq);
+  for (long t = tid; t < n4; t += nthreads) {
+    const float4 v = src[t];
+    dst[t] = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+  }
+}
+
+// ------------------------------------------------------------ main kernel
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(448, 1)
+    fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                  const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
+                  const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
+  uint64_t *bar_kv = bars + 0;
+  uint64_t *bar_qdo_full = bars + 1;   // [2]
+  uint64_t *bar_qdo_empty = bars + 3;  // [2]
+  uint64_t *bar_s_full = bars + 5;
+  uint64_t *bar_dp_full = bars + 6;
+  uint64_t *bar_p_full = bars + 7;
+  uint64_t *bar_ds_full = bars + 8;
+  uint64_t *bar_dv_done = bars + 9;
+  uint64_t *bar_dkq_done = bars + 10;
+  uint64_t *bar_dq_empty = bars + 11;
+  uint64_t *bar_epi = bars + 12;
+  uint64_t *bar_drain = bars + 13;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  uint8_t *sK = smem + C::kOffK;
+  uint8_t *sV = smem + C::kOffV;
+  uint8_t *sQ = smem + C::kOffQ;
+  uint8_t *sdO = smem + C::kOffdO;
+  uint8_t *sdS = smem + C::kOffdS;
+  float *sL = reinterpret_cast<float *>(smem + C::kOffL);
+  float *sDv = reinterpret_cast<float *>(smem + C::kOffDv);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x % p.BH;
+  const int j = blockIdx.x / p.BH;  // key tile; small j first (longest first when causal)
+  const int nq = (p.N + 127) / 128;
+  const int i0 = CAUSAL ? j : 0;
+  const int n_it = nq - i0;
+
+  const WaitCtx ctx{p.status, abort_flag, kKernelBwd, p.seq};
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    if ((smem_u32(smem) & 1023u) != 0) record_failure(ctx, kStatusInternal, 0);
+    mbar_init(bar_kv, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar_qdo_full[s], 1);
+      mbar_init(&bar_qdo_empty[s], 1);
+    }
+    mbar_init(bar_s_full, 1);
+    mbar_init(bar_dp_full, 1);
+    mbar_init(bar_p_full, 256);
+    mbar_init(bar_ds_full, 256);
+    mbar_init(bar_dv_done, 1);
+    mbar_init(bar_dkq_done, 1);
+    mbar_init(bar_dq_empty, 128);
+    mbar_init(bar_epi, 256);
+    mbar_init(bar_drain, 1);
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 13) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 12) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && !*abort_flag) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmdO);
+      mbar_arrive_expect_tx(bar_kv, 2 * C::kTile);
+      for (int b = 0; b < C::kBoxes; ++b) {
+        tma_load_3d(&tmK, bar_kv, sK + b * 16384, b * 64, j * 128, bh);
+        tma_load_3d(&tmV, bar_kv, sV + b * 16384, b * 64, j * 128, bh);
+      }
+      bool ok = true;
+      int it = 0;
+      for (; it < n_it; ++it) {
+        const int s = it & 1, n = it >> 1;
+        if (n > 0 && !mbar_wait(ctx, &bar_qdo_empty[s], (n - 1) & 1, kBTagQdoEmpty)) {
+          ok = false;
+          break;
+        }
+        const int i = i0 + it;
+        mbar_arrive_expect_tx(&bar_qdo_full[s], 2 * C::kTile + 1024);
+        for (int b = 0; b < C::kBoxes; ++b) {
+          tma_load_3d(&tmQ, &bar_qdo_full[s], sQ + s * C::kTile + b * 16384, b * 64, i * 128, bh);
+          tma_load_3d(&tmdO, &bar_qdo_full[s], sdO + s * C::kTile + b * 16384, b * 64, i * 128, bh);
+        }
+        const size_t soff = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(i) * 128;
+        bulk_load_1d(sL + s * 128, p.ws_lse2 + soff, 512, &bar_qdo_full[s]);
+        bulk_load_1d(sDv + s * 128, p.ws_D + soff, 512, &bar_qdo_full[s]);
+      }
+      if (!ok) {
+        mbar_drain(bar_kv, 0);
+        for (int s = 0; s < 2 && s < it; ++s) {
+          const int last = s + ((it - 1 - s) / 2) * 2;
+          mbar_drain(&bar_qdo_full[s], (last >> 1) & 1);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 13) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && !*abort_flag) {
+      constexpr uint32_t id_ss = make_idesc_bf16(128, 128, 0, 0);     // S^T, dP^T
+      constexpr uint32_t id_kxmn = make_idesc_bf16(128, D, 0, 1);     // dV (A in TMEM), dK
+      constexpr uint32_t id_mnmn = make_idesc_bf16(128, D, 1, 1);     // dQ
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), adS = smem_u32(sdS);
+      const uint32_t tS = tmem + C::kColS, tdP = tmem + C::kColdP, tdK = tmem + C::kColdK;
+      const uint32_t tdV = tmem + C::kColdV, tdQ = tmem + C::kColdQ;
+      bool ok = mbar_wait(ctx, bar_kv, 0, kBTagKV);
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int s = it & 1, n = it >> 1;
+        const uint32_t aQ = smem_u32(sQ + s * C::kTile), adO = smem_u32(sdO + s * C::kTile);
+        ok = mbar_wait(ctx, &bar_qdo_full[s], n & 1, kBTagQdoFull);
+        if (ok && it > 0) ok = mbar_wait(ctx, bar_dv_done, (it - 1) & 1, kBTagDvDone);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          mma_ss(tS, make_sdesc(aK + off, 16, 1024), make_sdesc(aQ + off, 16, 1024), id_ss, ks > 0);
+        }
+        mma_commit(bar_s_full);
+        if (D == 128 && it > 0) {
+          ok = mbar_wait(ctx, bar_dq_empty, (it - 1) & 1, kBTagDqEmpty);
+          if (!ok) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          mma_ss(tdP, make_sdesc(aV + off, 16, 1024), make_sdesc(adO + off, 16, 1024), id_ss, ks > 0);
+        }
+        mma_commit(bar_dp_full);
+        ok = mbar_wait(ctx, bar_p_full, it & 1, kBTagPFull);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ts(tdV, tS + ks * 8, make_sdesc(adO + ks * 2048, 16384, 1024), id_kxmn, (it > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(bar_dv_done);
+        ok = mbar_wait(ctx, bar_ds_full, it & 1, kBTagDsFull);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          mma_ss(tdK, make_sdesc(adS + off, 16, 1024), make_sdesc(aQ + ks * 2048, 16384, 1024), id_kxmn,
+                 (it > 0 || ks > 0) ? 1u : 0u);
+        }
+        if (D == 64 && it > 0) {
+          ok = mbar_wait(ctx, bar_dq_empty, (it - 1) & 1, kBTagDqEmpty);
+          if (!ok) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ss(tdQ, make_sdesc(adS + ks * 2048, 16384, 1024), make_sdesc(aK + ks * 2048, 16384, 1024), id_mnmn,
+                 ks > 0);
+        mma_commit(bar_dkq_done);
+        mma_commit(&bar_qdo_empty[s]);
+      }
+      if (!ok) {
+        mma_commit(bar_drain);
+        mbar_drain(bar_drain, 0);
+      }
+    }
+    __syncwarp();
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ compute
+    const int w = warp >> 2;                 // query-column half
+    const int r = (warp & 3) * 32 + lane;    // key row within the tile == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::kColS;
+    const uint32_t tdP = tmem + lane_off + C::kColdP;
+    const uint32_t dS_addr = smem_u32(sdS) + w * 16384;
+    const float c = p.scale_log2;
+    bool ok = !*abort_flag;
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int s = it & 1, n = it >> 1;
+      const int i = i0 + it;
+      ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_s_full, it & 1, kBTagSFull) &&
+                                       mbar_wait(ctx, &bar_qdo_full[s], n & 1, kBTagQdoFull));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[64];
+      tmem_ld32(tS + 64 * w, sv);
+      tmem_ld32(tS + 64 * w + 32, sv + 32);
+      tmem_wait_ld();
+      const float *lse2 = sL + s * 128 + 64 * w;
+      float pf[64];
+#pragma unroll
+      for (int cc = 0; cc < 64; ++cc) pf[cc] = ex2(fmaf(__uint_as_float(sv[cc]), c, -lse2[cc]));
+      if (CAUSAL && i == j) {
+        // Diagonal tile: key row r is masked for query columns before it.
+#pragma unroll
+        for (int cc = 0; cc < 64; ++cc)
+          if (64 * w + cc < r) pf[cc] = 0.f;
+      }
+      uint32_t pk[32];
+#pragma unroll
+      for (int t = 0; t < 32; ++t) pk[t] = pack_bf16(pf[2 * t], pf[2 * t + 1]);
+      tmem_st32(tS + 32 * w, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_p_full);
+
+      ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dp_full, it & 1, kBTagDpFull));
+      // The previous tile's dK / dQ MMAs read dS from smem: wait until they are done.
+      if (ok && it > 0) ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, (it - 1) & 1, kBTagDkqDone));
+      if (!ok) break;
+      tc_fence_after();
+      const float *Dv = sDv + s * 128 + 64 * w;
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t dp[32];
+        tmem_ld32(tdP + 64 * w + 32 * ch, dp);
+        tmem_wait_ld();
+        uint32_t dsk[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const int c0 = 32 * ch + 2 * t;
+          const float d0 = pf[c0] * (__uint_as_float(dp[2 * t]) - Dv[c0]);
+          const float d1 = pf[c0 + 1] * (__uint_as_float(dp[2 * t + 1]) - Dv[c0 + 1]);
+          dsk[t] = pack_bf16(d0, d1);
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          st_shared_v4(dS_addr + bsw128(r, 4 * ch + t), dsk[4 * t], dsk[4 * t + 1], dsk[4 * t + 2], dsk[4 * t + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_ds_full);
+    }
+    // ---------------------------------------------------------- epilogue
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, (n_it - 1) & 1, kBTagDkqDone));
+    if (ok) {
+      tc_fence_after();
+      // Every MMA has completed and every load was consumed: stage dV in the
+      // Q buffers and dK in the dO buffers.
+      const uint32_t stV = smem_u32(sQ), stK = smem_u32(sdO);
+      const uint32_t tdK = tmem + lane_off + C::kColdK, tdV = tmem + lane_off + C::kColdV;
+#pragma unroll
+      for (int ch = 0; ch < D / 64; ++ch) {
+        const int col0 = w * (D / 2) + 32 * ch;  // first feature of this 32-column chunk
+        const int box = col0 / 64, chunk0 = (col0 % 64) / 8;
+        uint32_t a[32], pkv[16];
+        tmem_ld32(tdV + col0, a);
+        tmem_wait_ld();
+#pragma unroll
+        for (int t = 0; t < 16; ++t) pkv[t] = pack_bf16(__uint_as_float(a[2 * t]), __uint_as_float(a[2 * t + 1]));
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          st_shared_v4(stV + box * 16384 + bsw128(r, chunk0 + t), pkv[4 * t], pkv[4 * t + 1], pkv[4 * t + 2],
+                       pkv[4 * t + 3]);
+        tmem_ld32(tdK + col0, a);
+        tmem_wait_ld();
+#pragma unroll
+        for (int t = 0; t < 16; ++t)
+          pkv[t] = pack_bf16(__uint_as_float(a[2 * t]) * p.scale, __uint_as_float(a[2 * t + 1]) * p.scale);
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          st_shared_v4(stK + box * 16384 + bsw128(r, chunk0 + t), pkv[4 * t], pkv[4 * t + 1], pkv[4 * t + 2],
+                       pkv[4 * t + 3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar_epi);
+      if (threadIdx.x == 0 && mbar_wait(ctx, bar_epi, 0, kBTagEpi)) {
+        for (int b = 0; b < C::kBoxes; ++b) {
+          tma_store_3d(&tmdV, sQ + b * 16384, b * 64, j * 128, bh);
+          tma_store_3d(&tmdK, sdO + b * 16384, b * 64, j * 128, bh);
+        }
+        bulk_commit();
+        bulk_wait_read<0>();
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ dQ drain
+    const int r = (warp & 3) * 32 + lane;  // query row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tdQ = tmem + lane_off + C::kColdQ;
+    bool ok = !*abort_flag;
+    for (int it = 0; it < n_it && ok; ++it) {
+      ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, it & 1, kBTagDkqDone));
+      if (!ok) break;
+      tc_fence_after();
+      const int qrow = (i0 + it) * 128 + r;
+      float *dst = p.ws_dq + (static_cast<size_t>(bh) * p.N + (qrow < p.N ? qrow : 0)) * D;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t v[32];
+        tmem_ld32(tdQ + 32 * ch, v);
+        tmem_wait_ld();
+        if (qrow < p.N) {
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            red_add_v4(dst + 32 * ch + 4 * t, __uint_as_float(v[4 * t]) * p.scale,
+                       __uint_as_float(v[4 * t + 1]) * p.scale, __uint_as_float(v[4 * t + 2]) * p.scale,
+                       __uint_as_float(v[4 * t + 3]) * p.scale);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_dq_empty);
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 13) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------ host side
+inline int pad128(int n) { return (n + 127) / 128 * 128; }
+
+inline size_t bwd_workspace_bytes(int BH, int N, int d) {
+  const size_t dq = static_cast<size_t>(BH) * N * d * 4;
+  const size_t vec = static_cast<size_t>(BH) * pad128(N) * 4;
+  const size_t total = dq + 2 * vec;
+  return (total + 255) / 256 * 256;
+}
+
+struct BwdLaunch {
+  const void *q, *k, *v, *o, *dO;
+  const float *lse;
+  void *dq, *dk, *dv;
+  int BH, N, d, causal;
+  float scale;
+  void *workspace;
+  int *status;
+  int seq;
+  int num_sms;
+  cudaEvent_t const *events = nullptr;  // optional: 4 events recorded around the stages
+};
+
+inline cudaError_t bwd_set_attributes() {
+  cudaError_t e = cudaFuncSetAttribute(fa_bwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       BwdCfg<64>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fa_bwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             BwdCfg<64>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fa_bwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             BwdCfg<128>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fa_bwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             BwdCfg<128>::kSmemBytes);
+  return e;
+}
+
+template <int D, bool CAUSAL>
+inline void bwd_main_launch(const CUtensorMap *m, const BwdParams &p, int nkv, cudaStream_t s) {
+  const dim3 grid(static_cast<unsigned>(p.BH) * static_cast<unsigned>(nkv));
+  fa_bwd_kernel<D, CAUSAL><<<grid, BwdCfg<D>::kThreads, BwdCfg<D>::kSmemBytes, s>>>(m[0], m[1], m[2], m[3], m[4],
+                                                                                      m[5], p);
+}
+
+// maps: Q, K, V, dO, dK, dV (bf16, 3-D, 64-feature boxes).
+inline cudaError_t bwd_launch(const BwdLaunch &L, const CUtensorMap *maps, cudaStream_t s) {
+  const int Npad = pad128(L.N);
+  float *ws_dq = static_cast<float *>(L.workspace);
+  float *ws_lse2 = ws_dq + static_cast<size_t>(L.BH) * L.N * L.d;
+  float *ws_D = ws_lse2 + static_cast<size_t>(L.BH) * Npad;
+  const int pre_grid = L.num_sms * 4;
+  cudaError_t e = cudaSuccess;
+  if (L.events && (e = cudaEventRecord(L.events[0], s)) != cudaSuccess) return e;
+  if (L.d == 64)
+    fa_bwd_pre_kernel<64><<<pre_grid, 256, 0, s>>>(static_cast<const uint16_t *>(L.o),
+                                                   static_cast<const uint16_t *>(L.dO), L.lse, ws_D, ws_lse2, ws_dq,
+                                                   L.N, Npad, L.BH);
+  else
+    fa_bwd_pre_kernel<128><<<pre_grid, 256, 0, s>>>(static_cast<const uint16_t *>(L.o),
+                                                    static_cast<const uint16_t *>(L.dO), L.lse, ws_D, ws_lse2, ws_dq,
+                                                    L.N, Npad, L.BH);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (L.events && (e = cudaEventRecord(L.events[1], s)) != cudaSuccess) return e;
+  BwdParams p;
+  p.ws_lse2 = ws_lse2;
+  p.ws_D = ws_D;
+  p.ws_dq = ws_dq;
+  p.status = L.status;
+  p.seq = L.seq;
+  p.N = L.N;
+  p.Npad = Npad;
+  p.BH = L.BH;
+  p.scale_log2 = L.scale * 1.4426950408889634f;
+  p.scale = L.scale;
+  const int nkv = Npad / 128;
+  if (L.d == 64)
+    L.causal ? bwd_main_launch<64, true>(maps, p, nkv, s) : bwd_main_launch<64, false>(maps, p, nkv, s);
+  else
+    L.causal ? bwd_main_launch<128, true>(maps, p, nkv, s) : bwd_main_launch<128, false>(maps, p, nkv, s);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (L.events && (e = cudaEventRecord(L.events[2], s)) != cudaSuccess) return e;
+  const long n4 = static_cast<long>(L.BH) * L.N * L.d / 4;
+  fa_dq_convert_kernel<<<L.num_sms * 4, 256, 0, s>>>(ws_dq, static_cast<uint16_t *>(L.dq), n4);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (L.events) e = cudaEventRecord(L.events[3], s);
+  return e;
+}
+
+}  // namespace fa

@@ -50,7 +50,9 @@ def _load():
         lib.ref_attn_bwd.argtypes = [D, D, D, D, D, D, D, cl, cl, cl, cl, cd, ci, ci]
         lib.ref_attn_fwd_rows.argtypes = [D, D, D, cl, cl, cl, cl, cd, ci, L, L, cl, D, D, ci]
         lib.ref_attn_dq_rows.argtypes = [D, D, D, D, cl, cl, cl, cl, cd, ci, L, L, cl, D, ci]
-        for f in (lib.ref_attn_fwd, lib.ref_attn_bwd, lib.ref_attn_fwd_rows, lib.ref_attn_dq_rows):
+        lib.ref_attn_dkdv_rows.argtypes = [D, D, D, D, cl, cl, cl, cl, cd, ci, cl, L, cl, D, D, ci]
+        for f in (lib.ref_attn_fwd, lib.ref_attn_bwd, lib.ref_attn_fwd_rows, lib.ref_attn_dq_rows,
+                  lib.ref_attn_dkdv_rows):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -139,3 +141,20 @@ def ref_dq_rows(q, k, v, dO, scale: float, causal: bool, samp_bh, samp_row, nthr
     if rc != 0:
         raise RuntimeError(f"ref_attn_dq_rows failed ({rc})")
     return dq
+
+
+def ref_dkdv_rows(q, k, v, dO, scale: float, causal: bool, head: int, key_rows, nthreads: int = 0):
+    """dK, dV rows [n, d] of one head (flat index) at the given key rows."""
+    q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
+    B, H, N, d = _shape4(q)
+    kr = np.ascontiguousarray(np.asarray(key_rows, dtype=np.int64)).astype(np.dtype("l"))
+    n = kr.shape[0]
+    dk = np.empty((n, d), dtype=np.float64)
+    dv = np.empty((n, d), dtype=np.float64)
+    Lp = ctypes.POINTER(ctypes.c_long)
+    rc = _load().ref_attn_dkdv_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), B, H, N, d, float(scale),
+                                    int(bool(causal)), int(head), kr.ctypes.data_as(Lp), n,
+                                    _ptr(dk), _ptr(dv), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"ref_attn_dkdv_rows failed ({rc})")
+    return dk, dv

@@ -179,7 +179,8 @@ static void bwd_col(const double *q, const double *k, const double *v,
 /* ------------------------------------------------------------ thread pool */
 
 typedef struct {
-    int kind; /* 0 fwd rows, 1 bwd sweep 1, 2 bwd sweep 2, 3 sampled fwd, 4 sampled dq */
+    int kind; /* 0 fwd rows, 1 bwd sweep 1, 2 bwd sweep 2, 3 sampled fwd, 4 sampled dq,
+                 5 sweep 1 over query rows [row0, N) of one head, 6 sweep 2 at sampled key rows */
     const double *q, *k, *v, *dO;
     double *o, *lse, *dq, *dk, *dv;
     double *m, *l, *D;           /* [B*H*N] scratch for the backward */
@@ -188,6 +189,8 @@ typedef struct {
     long BH, N, d;
     double scale;
     int causal;
+    long row0;                   /* first query row (kind 5); head index (kinds 5, 6) */
+    long head;
     long chunk;                  /* rows per task */
     long n_tasks;
     atomic_long next;
@@ -196,6 +199,24 @@ typedef struct {
 static void run_task(job_t *J, long t, double *srow, double *dprow)
 {
     long N = J->N, d = J->d;
+    if (J->kind == 5 || J->kind == 6) {
+        long h = J->head;
+        const double *q = J->q + h * N * d, *k = J->k + h * N * d,
+                     *v = J->v + h * N * d, *dO = J->dO + h * N * d;
+        if (J->kind == 5) {
+            long r0 = J->row0 + t * J->chunk, r1 = r0 + J->chunk;
+            if (r1 > N)
+                r1 = N;
+            for (long r = r0; r < r1; ++r)
+                bwd_row(q, k, v, dO, N, d, J->scale, J->causal, r, J->m + r,
+                        J->l + r, J->D + r, J->dq + r * d, srow, dprow);
+        } else {
+            long j = J->samp_row[t];
+            bwd_col(q, k, v, dO, J->m, J->l, J->D, N, d, J->scale, J->causal,
+                    j, J->dk + t * d, J->dv + t * d);
+        }
+        return;
+    }
     if (J->kind == 3 || J->kind == 4) {
         long s0 = t * J->chunk, s1 = s0 + J->chunk;
         if (s1 > J->n_samples)
@@ -417,4 +438,53 @@ int ref_attn_dq_rows(const double *q, const double *k, const double *v,
     J.chunk = 1;
     J.n_tasks = n_samples;
     return run_job(&J, nthreads);
+}
+
+/* dK, dV at sampled key rows of one head (flat head index `head`): dk_s, dv_s
+ * [n, d].  Sweep 1 runs only over the query rows that can see those keys
+ * (rows >= min key row when causal, every row otherwise), so the cost for keys
+ * near the end of a causal sequence is small at any N. */
+int ref_attn_dkdv_rows(const double *q, const double *k, const double *v,
+                       const double *dO, long B, long H, long N, long d,
+                       double scale, int causal, long head,
+                       const long *key_rows, long n_keys, double *dk_s,
+                       double *dv_s, int nthreads)
+{
+    if (!q || !k || !v || !dO || !key_rows || !dk_s || !dv_s ||
+        bad_shape(B, H, N, d) || head < 0 || head >= B * H || n_keys < 0)
+        return -1;
+    long row0 = N;
+    for (long s = 0; s < n_keys; ++s) {
+        if (key_rows[s] < 0 || key_rows[s] >= N)
+            return -1;
+        if (key_rows[s] < row0)
+            row0 = key_rows[s];
+    }
+    if (n_keys == 0)
+        return 0;
+    if (!causal)
+        row0 = 0;
+    double *buf = (double *)malloc(sizeof(double) * (size_t)(N * (3 + d)));
+    if (!buf)
+        return -2;
+    job_t J;
+    memset(&J, 0, sizeof(J));
+    J.q = q; J.k = k; J.v = v; J.dO = dO;
+    J.m = buf; J.l = buf + N; J.D = buf + 2 * N; J.dq = buf + 3 * N;
+    J.dk = dk_s; J.dv = dv_s;
+    J.samp_row = key_rows; J.n_samples = n_keys;
+    J.BH = B * H; J.N = N; J.d = d; J.scale = scale; J.causal = causal;
+    J.head = head; J.row0 = row0;
+    J.kind = 5;
+    J.chunk = pick_chunk(1, N - row0, nthreads);
+    J.n_tasks = (N - row0 + J.chunk - 1) / J.chunk;
+    int rc = run_job(&J, nthreads);
+    if (rc == 0) {
+        J.kind = 6;
+        J.chunk = 1;
+        J.n_tasks = n_keys;
+        rc = run_job(&J, nthreads);
+    }
+    free(buf);
+    return rc;
 }

@@ -354,6 +354,22 @@ def test_sampled_rows_match_full(causal):
     assert close(dqs, dqf[sb, sr], 1e-13)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampled_key_rows_match_full(causal):
+    B, H, N, d = 1, 3, 45, 8
+    q, k, v, dO = (rnd((B, H, N, d), 80 + s) for s in range(4))
+    _, dk, dv = c_bwd(q, k, v, dO, 0.3, causal)
+    for head in (0, 2):
+        keys = np.array([44, 3, 20, 43, 0])
+        dks, dvs = oracle.ref_dkdv_rows(q, k, v, dO, 0.3, causal, head, keys)
+        assert close(dks, dk.reshape(B * H, N, d)[head, keys], 1e-12)
+        assert close(dvs, dv.reshape(B * H, N, d)[head, keys], 1e-12)
+    tail = np.arange(40, 45)
+    dks, dvs = oracle.ref_dkdv_rows(q, k, v, dO, 0.3, causal, 1, tail)
+    assert close(dks, dk.reshape(B * H, N, d)[1, tail], 1e-12)
+    assert close(dvs, dv.reshape(B * H, N, d)[1, tail], 1e-12)
+
+
 def test_thread_count_does_not_change_forward():
     q, k, v = (rnd((1, 2, 64, 8), 70 + s) for s in range(3))
     o1, l1 = oracle.ref_fwd(q, k, v, 0.3, True, nthreads=1)

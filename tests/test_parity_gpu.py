@@ -1,0 +1,186 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Every input comes from the seeded generator (io_aware_exact_23_b200.inputs);
+every expected value comes from ``oracle``.  Small shapes are compared element
+by element over whole tensors; the full-size workloads are compared at sampled
+(head, row) positions the oracle computes one by one (O, LSE, dQ rows; dK, dV
+rows at the key tiles whose query stats are cheap), plus gradient identities
+that hold at any size:  sum_j dK_j = 0,  sum_j dV_j = sum_i dO_i  and
+sum_i Q_i.dQ_i = sum_j K_j.dK_j.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from io_aware_exact_23_b200 import inputs as I
+from io_aware_exact_23_b200.inputs import Workload, make_inputs
+
+from gpu_helpers import (TOL_GRAD_REL, TOL_LSE, TOL_O, full_check, gpu_backward, gpu_forward, max_err,
+                         sample_rows, to64)
+
+pytestmark = pytest.mark.gpu
+
+
+# ------------------------------------------------------------ small, full
+def test_tiny_config_full():
+    full_check(I.TINY)
+
+
+EDGE = [(n, d, c) for d in (64, 128) for c in (False, True) for n in (1, 17, 128, 129, 255, 257, 300)]
+
+
+@pytest.mark.parametrize("N,d,causal", EDGE, ids=lambda x: str(x))
+def test_ragged_and_edge_lengths_full(N, d, causal):
+    full_check(Workload(f"edge_n{N}", 1, 2, N, d, causal, seed=N))
+
+
+@pytest.mark.parametrize("d,causal", [(64, False), (64, True), (128, False), (128, True)])
+def test_multi_head_ragged_full(d, causal):
+    full_check(Workload("mh", 2, 3, 1000, d, causal, seed=7))
+
+
+@pytest.mark.parametrize("d,causal", [(64, False), (64, True), (128, False), (128, True)])
+def test_stress_x8_full(d, causal):
+    """Q, K x 8: logits with std ~ 64 (near one-hot rows, frequent max updates)."""
+    full_check(Workload("stress", 1, 2, 768, d, causal, qk_mult=8.0, seed=3))
+
+
+# ------------------------------------------------------------ exactness
+def test_causal_row0_is_v0_exactly():
+    w = Workload("row0", 2, 4, 512, 128, True, seed=11)
+    t = make_inputs(w, device="cuda")
+    o, _ = gpu_forward(t, w.scale, True)
+    assert torch.equal(o[:, :, 0], t["v"][:, :, 0])
+
+
+def test_forward_is_deterministic():
+    w = Workload("det", 2, 4, 1024, 64, False, seed=12)
+    t = make_inputs(w, device="cuda")
+    o1, l1 = gpu_forward(t, w.scale, False)
+    o2, l2 = gpu_forward(t, w.scale, False)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_outputs_stay_inside_their_buffers():
+    """Guard bands of NaN around every output are left untouched."""
+    from io_aware_exact_23_b200 import binding as fa
+    w = Workload("guard", 1, 3, 300, 128, True, seed=13)
+    t = make_inputs(w, device="cuda")
+    n = w.elems()
+    G = 4096  # guard elements on each side (16-byte multiples keep alignment)
+
+    def guarded(numel, dtype):
+        buf = torch.full((numel + 2 * G,), float("nan"), dtype=dtype, device="cuda")
+        return buf, buf[G:G + numel]
+
+    ob, o = guarded(n, torch.bfloat16)
+    lb, lse = guarded(w.B * w.H * w.N, torch.float32)
+    o, lse = o.view(t["q"].shape), lse.view(w.B, w.H, w.N)
+    fa.fa_fwd(t["q"], t["k"], t["v"], o, lse, w.scale, True)
+    grads = [guarded(n, torch.bfloat16) for _ in range(3)]
+    ws = torch.zeros(fa.fa_bwd_workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device="cuda")
+    fa.fa_bwd(t["q"], t["k"], t["v"], o, t["do"], lse, *(g[1].view(t["q"].shape) for g in grads), w.scale,
+              True, ws)
+    assert fa.fa_device_status() == 0
+    for buf in [ob, lb] + [g[0] for g in grads]:
+        assert torch.isnan(buf[:G].float()).all() and torch.isnan(buf[-G:].float()).all()
+    for x in [o, lse] + [g[1] for g in grads]:
+        assert torch.isfinite(x.float()).all()
+
+
+def test_argument_error_touches_nothing():
+    from io_aware_exact_23_b200 import binding as fa
+    L = fa.lib()
+    q = torch.randn(1, 1, 256, 64, device="cuda").to(torch.bfloat16)
+    o = torch.full_like(q, 7.0)
+    lse = torch.full((1, 1, 256), 7.0, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    assert L.fa_fwd(q.data_ptr(), q.data_ptr(), q.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                    1, 1, 256, 96, 0.1, 0, s) == 2
+    assert L.fa_fwd(q.data_ptr(), q.data_ptr(), q.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                    1, 1, 256, 64, float("nan"), 0, s) == 1
+    assert L.fa_fwd(q.data_ptr() + 2, q.data_ptr(), q.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                    1, 1, 256, 64, 0.1, 0, s) == 3
+    torch.cuda.synchronize()
+    assert (o == 7.0).all() and (lse == 7.0).all()
+    assert fa.fa_device_status() == 0
+
+
+def test_non_default_stream():
+    w = Workload("stream", 1, 4, 640, 64, True, seed=14)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        t = make_inputs(w, device="cuda")
+        o, lse = gpu_forward(t, w.scale, True)
+    o_ref, l_ref = oracle.ref_fwd(t["q"], t["k"], t["v"], w.scale, True)
+    assert max_err(to64(o), o_ref) <= TOL_O and max_err(to64(lse), l_ref) <= TOL_LSE
+
+
+# ------------------------------------------------------ full-size workloads
+def check_sampled(w: Workload, n_rows=192, dkdv_full_head_max_n=4096, n_tail_keys=128):
+    t = make_inputs(w, device="cuda")
+    o, lse = gpu_forward(t, w.scale, w.causal)
+    dq, dk, dv = gpu_backward(t, o, lse, w.scale, w.causal)
+    BH, N, d = w.B * w.H, w.N, w.d
+    sb, sr = sample_rows(BH, N, n_rows, seed=w.N + d)
+    o_ref, l_ref = oracle.ref_fwd_rows(t["q"], t["k"], t["v"], w.scale, w.causal, sb, sr)
+    of, lf = to64(o).reshape(BH, N, d), to64(lse).reshape(BH, N)
+    eo, el = max_err(of[sb, sr], o_ref), max_err(lf[sb, sr], l_ref)
+    assert eo <= TOL_O, f"{w.name}: sampled max|O-O_ref| = {eo:.3e}"
+    assert el <= TOL_LSE, f"{w.name}: sampled max|LSE-LSE_ref| = {el:.3e}"
+    # dQ at the same rows; the gate's scale is the oracle's max over the sampled rows
+    dq_ref = oracle.ref_dq_rows(t["q"], t["k"], t["v"], t["do"], w.scale, w.causal, sb, sr)
+    dqf = to64(dq).reshape(BH, N, d)
+    e = max_err(dqf[sb, sr], dq_ref)
+    assert e <= TOL_GRAD_REL * np.abs(dq_ref).max(), f"{w.name}: sampled dQ err {e:.3e}"
+    # dK, dV rows: a whole head when affordable, else the last key tile(s) of a
+    # causal head (their query statistics only need the last rows).
+    dkf, dvf = to64(dk).reshape(BH, N, d), to64(dv).reshape(BH, N, d)
+    head = int(np.random.default_rng(w.N).integers(0, BH))
+    if N <= dkdv_full_head_max_n:
+        keys = np.arange(N)
+    elif w.causal:
+        keys = np.arange(N - n_tail_keys, N)
+    else:
+        keys = None
+    if keys is not None:
+        rk, rv = oracle.ref_dkdv_rows(t["q"], t["k"], t["v"], t["do"], w.scale, w.causal, head, keys)
+        for nm, g, r in (("dK", dkf[head, keys], rk), ("dV", dvf[head, keys], rv)):
+            e = max_err(g, r)
+            assert e <= TOL_GRAD_REL * np.abs(r).max(), f"{w.name}: {nm} err {e:.3e} vs {np.abs(r).max():.3e}"
+    # identities over every head, in fp64 on the GPU outputs
+    q64 = t["q"].double()
+    k64 = t["k"].double()
+    dk64, dv64, dq64 = dk.double(), dv.double(), dq.double()
+    s_dk = dk64.sum(2)
+    bound_dk = TOL_GRAD_REL * dk64.abs().amax(dim=(2, 3), keepdim=False) * np.sqrt(N)
+    assert (s_dk.abs().amax(dim=2) <= bound_dk + 1e-6).all(), f"{w.name}: sum_j dK_j != 0"
+    s_dv = dv64.sum(2) - t["do"].double().sum(2)
+    bound_dv = TOL_GRAD_REL * dv64.abs().amax(dim=(2, 3)) * np.sqrt(N)
+    assert (s_dv.abs().amax(dim=2) <= bound_dv + 1e-6).all(), f"{w.name}: sum_j dV_j != sum_i dO_i"
+    lhs = (q64 * dq64).sum((2, 3))
+    rhs = (k64 * dk64).sum((2, 3))
+    mag = (q64.abs() * dq64.abs()).sum((2, 3)) + (k64.abs() * dk64.abs()).sum((2, 3))
+    assert ((lhs - rhs).abs() <= TOL_GRAD_REL * mag).all(), f"{w.name}: sum Q.dQ != sum K.dK"
+    return {"o": eo, "lse": el}
+
+
+@pytest.mark.parametrize("w", [I.C2, I.C3], ids=lambda w: w.name)
+def test_full_size_configs(w):
+    check_sampled(w)
+
+
+@pytest.mark.slow
+def test_long_context_config():
+    check_sampled(I.C4, n_rows=96)
+
+
+SWEEP = I.sweep()
+
+
+@pytest.mark.parametrize("w", SWEEP, ids=lambda w: w.name)
+def test_sweep_point(w):
+    check_sampled(w, n_rows=64, dkdv_full_head_max_n=1024)
