@@ -94,18 +94,38 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o,
            void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * fa_bwd with stage timing.  `events` is either NULL (then this is exactly
- * fa_bwd) or a host array of four cudaEvent_t handles owned by the caller;
- * they are recorded on `stream` before the preprocess kernel, after it, after
- * the main dK/dV/dQ kernel, and after the dQ conversion, so the caller can time
- * each kernel with cudaEventElapsedTime.  Same arguments, layout and errors as
- * fa_bwd; FA_ERR_CUDA if recording an event fails.
+ * Forward pass that also writes the rounding residual of O:
+ *   o_lo [B,H,N,d] bf16 = bf16(O_fp32 - o),
+ * i.e. what rounding the fp32 result to the bf16 output o dropped, so that
+ * o + o_lo carries about 16 significant bits of O.  The backward's
+ * D_i = rowsum(dO_i o O_i) is a difference-sensitive quantity: in rows where
+ * softmax is nearly one-hot, dS = P (dP - D) cancels almost exactly and an
+ * 8-bit O would dominate the gradient error.  Passing o_lo to fa_bwd_ex
+ * removes that error.  o_lo must not overlap any other tensor; NULL makes
+ * this call identical to fa_fwd.  This is not a step of the pages' method but
+ * a precision choice of this implementation (the pages leave the backward's
+ * arithmetic open).
  */
-int fa_bwd_profiled(const void *q, const void *k, const void *v, const void *o,
-                    const void *dO, const float *lse, void *dq, void *dk,
-                    void *dv, int B, int H, int N, int d, float scale,
-                    int causal, void *workspace, size_t workspace_bytes,
-                    void *stream, void *const *events);
+int fa_fwd_residual(const void *q, const void *k, const void *v, void *o,
+                    void *o_lo, float *lse, int B, int H, int N, int d,
+                    float scale, int causal, void *stream);
+
+/*
+ * Backward pass with the optional extras:
+ *   o_lo    NULL, or the residual written by fa_fwd_residual (then
+ *           D_i = rowsum(dO o (o + o_lo)) instead of rowsum(dO o o));
+ *   events  NULL, or a host array of four cudaEvent_t handles owned by the
+ *           caller, recorded on `stream` before the preprocess kernel, after
+ *           it, after the main dK/dV/dQ kernel and after the dQ conversion, so
+ *           each kernel can be timed with cudaEventElapsedTime.
+ * Otherwise the same arguments, layout and errors as fa_bwd (FA_ERR_INVALID_ARG
+ * if an event handle is NULL, FA_ERR_CUDA if recording one fails).
+ */
+int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o,
+              const void *o_lo, const void *dO, const float *lse, void *dq,
+              void *dk, void *dv, int B, int H, int N, int d, float scale,
+              int causal, void *workspace, size_t workspace_bytes,
+              void *stream, void *const *events);
 
 /* Static, human-readable name of a status code (never NULL). */
 const char *fa_status_string(int status);

@@ -46,9 +46,11 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd.restype = i
         L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
         L.fa_bwd.restype = i
-        L.fa_bwd_profiled.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp,
-                                      ctypes.POINTER(vp)]
-        L.fa_bwd_profiled.restype = i
+        L.fa_fwd_residual.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+        L.fa_fwd_residual.restype = i
+        L.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp,
+                                ctypes.POINTER(vp)]
+        L.fa_bwd_ex.restype = i
         L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
         L.fa_bwd_workspace_bytes.restype = sz
         L.fa_status_string.argtypes = [i]
@@ -84,14 +86,24 @@ def _check(t: torch.Tensor, name: str, dtype, shape=None):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
-def fa_fwd(q, k, v, o, lse, scale: float, causal: bool, stream=None) -> None:
-    """O and LSE into the preallocated ``o`` [B,H,N,d] bf16 and ``lse`` [B,H,N] fp32."""
+def fa_fwd(q, k, v, o, lse, scale: float, causal: bool, stream=None, o_lo=None) -> None:
+    """O and LSE into the preallocated ``o`` [B,H,N,d] bf16 and ``lse`` [B,H,N] fp32.
+
+    ``o_lo``: optional bf16 tensor shaped like ``o`` that receives O's rounding
+    residual (``fa_fwd_residual``), for an exact backward ``D``.
+    """
     B, H, N, d = q.shape
     for nm, t in (("q", q), ("k", k), ("v", v), ("o", o)):
         _check(t, nm, torch.bfloat16, (B, H, N, d))
     _check(lse, "lse", torch.float32, (B, H, N))
-    rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                      B, H, N, d, float(scale), int(bool(causal)), _stream_handle(stream))
+    if o_lo is None:
+        rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                          B, H, N, d, float(scale), int(bool(causal)), _stream_handle(stream))
+    else:
+        _check(o_lo, "o_lo", torch.bfloat16, (B, H, N, d))
+        rc = lib().fa_fwd_residual(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), o_lo.data_ptr(),
+                                   lse.data_ptr(), B, H, N, d, float(scale), int(bool(causal)),
+                                   _stream_handle(stream))
     if rc != FA_OK:
         raise FaError(rc, "fa_fwd")
 
@@ -101,9 +113,10 @@ def fa_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
 
 
 def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, scale: float, causal: bool, workspace, stream=None,
-           events=None) -> None:
+           events=None, o_lo=None) -> None:
     """dQ, dK, dV into preallocated bf16 tensors; ``workspace`` is a uint8 CUDA tensor.
 
+    ``o_lo``: the residual from ``fa_fwd(..., o_lo=...)`` (optional).
     ``events``: optional sequence of four ``torch.cuda.Event(enable_timing=True)``
     recorded around the preprocess, main and dQ-conversion kernels.
     """
@@ -112,16 +125,26 @@ def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, scale: float, causal: bool, workspac
         _check(t, nm, torch.bfloat16, (B, H, N, d))
     _check(lse, "lse", torch.float32, (B, H, N))
     _check(workspace, "workspace", torch.uint8)
-    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dO.data_ptr(), lse.data_ptr(),
-            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, float(scale), int(bool(causal)),
-            workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
-    if events is None:
-        rc = lib().fa_bwd(*args)
+    if events is None and o_lo is None:
+        rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dO.data_ptr(), lse.data_ptr(),
+                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, float(scale),
+                          int(bool(causal)), workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
     else:
-        if len(events) != 4:
-            raise ValueError("events must hold four torch.cuda.Event objects")
-        handles = (ctypes.c_void_p * 4)(*[ev.cuda_event for ev in events])
-        rc = lib().fa_bwd_profiled(*args, handles)
+        handles = None
+        if events is not None:
+            if len(events) != 4:
+                raise ValueError("events must hold four torch.cuda.Event objects")
+            for ev in events:
+                if ev.cuda_event == 0:  # torch creates the CUDA event lazily, on first record
+                    ev.record()
+            handles = (ctypes.c_void_p * 4)(*[ev.cuda_event for ev in events])
+        if o_lo is not None:
+            _check(o_lo, "o_lo", torch.bfloat16, (B, H, N, d))
+        rc = lib().fa_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             None if o_lo is None else o_lo.data_ptr(), dO.data_ptr(), lse.data_ptr(),
+                             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, float(scale),
+                             int(bool(causal)), workspace.data_ptr(), workspace.numel(), _stream_handle(stream),
+                             handles)
     if rc != FA_OK:
         raise FaError(rc, "fa_bwd")
 
@@ -140,16 +163,18 @@ class Attention:
         self.scale = float(scale)
         self.causal = bool(causal)
 
-    def forward(self, q, k, v):
+    def forward(self, q, k, v, residual: bool = True):
+        """Returns (o, lse, o_lo); o_lo is None when ``residual`` is False."""
         B, H, N, d = q.shape
         o = torch.empty_like(q)
+        o_lo = torch.empty_like(q) if residual else None
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-        fa_fwd(q, k, v, o, lse, self.scale, self.causal)
-        return o, lse
+        fa_fwd(q, k, v, o, lse, self.scale, self.causal, o_lo=o_lo)
+        return o, lse, o_lo
 
-    def backward(self, q, k, v, o, lse, dO):
+    def backward(self, q, k, v, o, lse, dO, o_lo=None):
         B, H, N, d = q.shape
         ws = torch.empty(fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=q.device)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, self.scale, self.causal, ws)
+        fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, self.scale, self.causal, ws, o_lo=o_lo)
         return dq, dk, dv

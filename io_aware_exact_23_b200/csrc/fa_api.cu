@@ -182,12 +182,14 @@ const char *fa_status_string(int status) {
   }
 }
 
-int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N, int d,
-           float scale, int causal, void *stream) {
+int fa_fwd_residual(const void *q, const void *k, const void *v, void *o, void *o_lo, float *lse, int B, int H,
+                    int N, int d, float scale, int causal, void *stream) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   int st = check_shape(B, H, N, d, scale, causal);
   if (st != FA_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      (o_lo && !aligned16(o_lo)))
+    return FA_ERR_MISALIGNED;
   DeviceState *ds = nullptr;
   st = device_state(&ds, nullptr);
   if (st != FA_OK) return st;
@@ -199,6 +201,7 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
     return FA_ERR_CUDA;
   fa::FwdParams p;
   p.lse = lse;
+  p.o_lo = static_cast<uint16_t *>(o_lo);
   p.status = ds->status;
   p.seq = next_seq();
   p.N = N;
@@ -214,19 +217,24 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N, int d,
+           float scale, int causal, void *stream) {
+  return fa_fwd_residual(q, k, v, o, nullptr, lse, B, H, N, d, scale, causal, stream);
+}
+
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   if (check_shape(B, H, N, d, 1.f, 0) != FA_OK) return 0;
   return fa::bwd_workspace_bytes(B * H, N, d);
 }
 
-int fa_bwd_profiled(const void *q, const void *k, const void *v, const void *o, const void *dO,
-                    const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale,
-                    int causal, void *workspace, size_t workspace_bytes, void *stream, void *const *events) {
+int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o, const void *o_lo, const void *dO,
+              const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale, int causal,
+              void *workspace, size_t workspace_bytes, void *stream, void *const *events) {
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   int st = check_shape(B, H, N, d, scale, causal);
   if (st != FA_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) || !aligned16(lse) ||
-      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (o_lo && !aligned16(o_lo)))
     return FA_ERR_MISALIGNED;
   const int BH = B * H;
   if (!workspace || workspace_bytes < fa::bwd_workspace_bytes(BH, N, d)) return FA_ERR_WORKSPACE;
@@ -237,7 +245,7 @@ int fa_bwd_profiled(const void *q, const void *k, const void *v, const void *o, 
   if (st != FA_OK) return st;
 
   fa::BwdLaunch L;
-  L.q = q; L.k = k; L.v = v; L.o = o; L.dO = dO; L.lse = lse;
+  L.q = q; L.k = k; L.v = v; L.o = o; L.o_lo = o_lo; L.dO = dO; L.lse = lse;
   L.dq = dq; L.dk = dk; L.dv = dv;
   L.BH = BH; L.N = N; L.d = d; L.scale = scale; L.causal = causal;
   L.workspace = workspace;
@@ -257,8 +265,8 @@ int fa_bwd_profiled(const void *q, const void *k, const void *v, const void *o, 
 int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dO, const float *lse, void *dq,
            void *dk, void *dv, int B, int H, int N, int d, float scale, int causal, void *workspace,
            size_t workspace_bytes, void *stream) {
-  return fa_bwd_profiled(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes,
-                         stream, nullptr);
+  return fa_bwd_ex(q, k, v, o, nullptr, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace,
+                   workspace_bytes, stream, nullptr);
 }
 
 int fa_device_status_info(void *stream, int *info) {

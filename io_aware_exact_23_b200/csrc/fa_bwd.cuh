@@ -8,7 +8,8 @@
 //   dQ = scale * dS K,  dK = scale * dS^T Q.
 //
 // Three kernels on one stream:
-//   1. fa_bwd_pre_kernel   D_i = rowsum(dO o O) and LSE_i*log2(e) into the
+//   1. fa_bwd_pre_kernel   D_i = rowsum(dO o O) (O = o + o_lo when the forward
+//                          wrote its rounding residual) and LSE_i*log2(e) into the
 //                          workspace (padded to whole 128-row tiles), and zero
 //                          the fp32 dQ accumulator.
 //   2. fa_bwd_kernel       one CTA per (head, 128-row key tile j): K_j, V_j stay
@@ -84,6 +85,7 @@ __device__ __forceinline__ uint32_t bsw128(int row, int chunk) {
 // Lanes-per-row = D / 8 (each lane handles 8 features = 16 bytes).
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t *__restrict__ o,
+                                                         const uint16_t *__restrict__ o_lo,
                                                          const uint16_t *__restrict__ dO,
                                                          const float *__restrict__ lse, float *__restrict__ ws_D,
                                                          float *__restrict__ ws_lse2, float *__restrict__ ws_dq,
@@ -111,6 +113,15 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t *__restr
       for (int t = 0; t < 4; ++t) {
         acc = fmaf(__uint_as_float(av[t] << 16), __uint_as_float(bv[t] << 16), acc);
         acc = fmaf(__uint_as_float(av[t] & 0xFFFF0000u), __uint_as_float(bv[t] & 0xFFFF0000u), acc);
+      }
+      if (o_lo != nullptr) {
+        const uint4 c = *reinterpret_cast<const uint4 *>(o_lo + off);
+        const uint32_t cv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          acc = fmaf(__uint_as_float(cv[t] << 16), __uint_as_float(bv[t] << 16), acc);
+          acc = fmaf(__uint_as_float(cv[t] & 0xFFFF0000u), __uint_as_float(bv[t] & 0xFFFF0000u), acc);
+        }
       }
     }
 #pragma unroll
@@ -477,7 +488,7 @@ inline size_t bwd_workspace_bytes(int BH, int N, int d) {
 }
 
 struct BwdLaunch {
-  const void *q, *k, *v, *o, *dO;
+  const void *q, *k, *v, *o, *o_lo, *dO;
   const float *lse;
   void *dq, *dk, *dv;
   int BH, N, d, causal;
@@ -522,10 +533,12 @@ inline cudaError_t bwd_launch(const BwdLaunch &L, const CUtensorMap *maps, cudaS
   if (L.events && (e = cudaEventRecord(L.events[0], s)) != cudaSuccess) return e;
   if (L.d == 64)
     fa_bwd_pre_kernel<64><<<pre_grid, 256, 0, s>>>(static_cast<const uint16_t *>(L.o),
+                                                   static_cast<const uint16_t *>(L.o_lo),
                                                    static_cast<const uint16_t *>(L.dO), L.lse, ws_D, ws_lse2, ws_dq,
                                                    L.N, Npad, L.BH);
   else
     fa_bwd_pre_kernel<128><<<pre_grid, 256, 0, s>>>(static_cast<const uint16_t *>(L.o),
+                                                    static_cast<const uint16_t *>(L.o_lo),
                                                     static_cast<const uint16_t *>(L.dO), L.lse, ws_D, ws_lse2, ws_dq,
                                                     L.N, Npad, L.BH);
   e = cudaGetLastError();

@@ -32,6 +32,7 @@ namespace fa {
 
 struct FwdParams {
   float *lse;        // [BH, N] fp32 (natural log)
+  uint16_t *o_lo;    // optional [BH, N, D] bf16: bf16(O_fp32 - O), or nullptr
   int *status;       // device status block
   int seq;           // launch sequence number (for the status block)
   int N;
@@ -329,6 +330,20 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int t = 0; t < 16; ++t)
           w[t] = pack_bf16(__uint_as_float(o[2 * t]) * inv_l, __uint_as_float(o[2 * t + 1]) * inv_l);
+        if (p.o_lo != nullptr && qt * 128 + r < p.N) {
+          // What rounding O to bf16 dropped, itself rounded to bf16: O ~ o + o_lo
+          // to about 16 significant bits (used by the backward's D = rowsum(dO o O)).
+          uint32_t lo[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const float a = __uint_as_float(o[2 * t]) * inv_l, b = __uint_as_float(o[2 * t + 1]) * inv_l;
+            lo[t] = pack_bf16(a - __uint_as_float(w[t] << 16), b - __uint_as_float(w[t] & 0xFFFF0000u));
+          }
+          uint4 *dst = reinterpret_cast<uint4 *>(p.o_lo + (static_cast<size_t>(bh) * p.N + qt * 128 + r) * D +
+                                                 ch * 32);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) dst[t] = make_uint4(lo[4 * t], lo[4 * t + 1], lo[4 * t + 2], lo[4 * t + 3]);
+        }
         const int box = ch >> 1;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
