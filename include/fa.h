@@ -127,6 +127,42 @@ int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o,
               int causal, void *workspace, size_t workspace_bytes,
               void *stream, void *const *events);
 
+/*
+ * Backward pass for callers that cannot allocate device memory.
+ *
+ * Some callers may not call cudaMalloc at all: code that runs where an
+ * allocation could block, fail or be forbidden (for example inside a memory
+ * pool or allocator of its own, in a real-time path with a fixed memory
+ * budget, or where device memory is handed out by a host framework that owns
+ * it).  This entry point computes exactly what fa_bwd computes, with the same
+ * arguments except the workspace: its scratch -- the fp32 dQ accumulator and
+ * the per-row D and LSE*log2(e) vectors -- lives in one static array of
+ * FA_NOALLOC_SCRATCH_BYTES bytes inside this library's device image.  Every
+ * GPU on which the library is loaded holds that array until the process exits.
+ * No counterpart exists in the pages; this is a deployment variant only.
+ *
+ * Limit: shapes whose scratch, fa_bwd_workspace_bytes(B, H, N, d), exceeds
+ * FA_NOALLOC_SCRATCH_BYTES are rejected with FA_ERR_WORKSPACE before anything
+ * is launched (e.g. at d = 128 about B*H*N <= 64 000 rows).
+ *
+ * The call allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ * library routine.  Its first call on a device does a one-time set-up on that
+ * device (it looks up the array's device address with cudaGetSymbolAddress and
+ * sets kernel attributes); make that first call before any stream capture.
+ * Every call shares the one array and each call re-initialises the part it
+ * uses (the dQ accumulator is zeroed by the first kernel of the call), so calls
+ * whose kernels overlap on the GPU -- on different streams, or from different
+ * host threads -- race on the array and must be serialised by the caller.
+ * A device-side wait timeout in these kernels is recorded in a status word that
+ * also lives in the static image; fa_device_status() does not see it (it owns
+ * a separately allocated word), and dq/dk/dv are then undefined.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                   const void *dO, const float *lse, void *dq, void *dk,
+                   void *dv, int B, int H, int N, int d, float scale,
+                   int causal, void *stream);
+
 /* Static, human-readable name of a status code (never NULL). */
 const char *fa_status_string(int status);
 

@@ -51,6 +51,8 @@ def lib() -> ctypes.CDLL:
         L.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp,
                                 ctypes.POINTER(vp)]
         L.fa_bwd_ex.restype = i
+        L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+        L.fa_bwd_noalloc.restype = i
         L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
         L.fa_bwd_workspace_bytes.restype = sz
         L.fa_status_string.argtypes = [i]
@@ -147,6 +149,26 @@ def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, scale: float, causal: bool, workspac
                              handles)
     if rc != FA_OK:
         raise FaError(rc, "fa_bwd")
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # FA_NOALLOC_SCRATCH_BYTES in include/fa.h
+
+
+def fa_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, scale: float, causal: bool, stream=None) -> None:
+    """``fa_bwd`` for callers that cannot allocate device memory: no workspace
+    argument; the scratch is a fixed static array inside libfa.so (shapes that
+    need more than NOALLOC_SCRATCH_BYTES are refused).  Calls that overlap on
+    the GPU share that array and race; the first call on a device does a
+    one-time set-up and should come before any stream capture."""
+    B, H, N, d = q.shape
+    for nm, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dO", dO), ("dq", dq), ("dk", dk), ("dv", dv)):
+        _check(t, nm, torch.bfloat16, (B, H, N, d))
+    _check(lse, "lse", torch.float32, (B, H, N))
+    rc = lib().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dO.data_ptr(),
+                              lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
+                              float(scale), int(bool(causal)), _stream_handle(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_bwd_noalloc")
 
 
 def fa_device_status(stream=None, info: bool = False):

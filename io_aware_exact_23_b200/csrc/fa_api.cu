@@ -300,3 +300,95 @@ int fa_device_status_info(void *stream, int *info) {
 int fa_device_status(void *stream) { return fa_device_status_info(stream, nullptr); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// fa_bwd_noalloc: fa_bwd for callers that cannot allocate device memory.  The
+// scratch it needs is this file-scope array in the library's device image.  In
+// host code the array's name is only a host-side stand-in, so its device
+// address is looked up once per device with cudaGetSymbolAddress (with that
+// device current) and passed to the kernels.
+static __device__ __align__(256) unsigned char fa_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+static __device__ __align__(256) int fa_noalloc_status[kStatusInts];
+
+namespace {
+
+struct NoAllocState {
+  bool ready = false;
+  void *scratch = nullptr;  // device address of fa_noalloc_scratch on this device
+  int *status = nullptr;    // device address of fa_noalloc_status on this device
+  int num_sms = 0;
+};
+
+NoAllocState g_noalloc[kMaxDevices];
+
+// One-time set-up on the current device; performs no allocation.
+int noalloc_state(NoAllocState **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    cudaGetLastError();
+    return FA_ERR_NO_DEVICE;
+  }
+  if (dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  NoAllocState &s = g_noalloc[dev];
+  if (!s.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_NO_DEVICE;
+    }
+    if (major != 10 || minor != 0) return FA_ERR_UNSUPPORTED;
+    void *scratch = nullptr, *status = nullptr;
+    if (cudaGetSymbolAddress(&scratch, fa_noalloc_scratch) != cudaSuccess ||
+        cudaGetSymbolAddress(&status, fa_noalloc_status) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    if (fa::bwd_set_attributes() != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    s.scratch = scratch;
+    s.status = static_cast<int *>(status);
+    s.num_sms = sms;
+    s.ready = true;
+  }
+  *out = &s;
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, const void *dO,
+                              const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d,
+                              float scale, int causal, void *stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  int st = check_shape(B, H, N, d, scale, causal);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_MISALIGNED;
+  const int BH = B * H;
+  if (fa::bwd_workspace_bytes(BH, N, d) > static_cast<size_t>(FA_NOALLOC_SCRATCH_BYTES)) return FA_ERR_WORKSPACE;
+  NoAllocState *ns = nullptr;
+  st = noalloc_state(&ns);
+  if (st != FA_OK) return st;
+
+  fa::BwdLaunch L;
+  L.q = q; L.k = k; L.v = v; L.o = o; L.o_lo = nullptr; L.dO = dO; L.lse = lse;
+  L.dq = dq; L.dk = dk; L.dv = dv;
+  L.BH = BH; L.N = N; L.d = d; L.scale = scale; L.causal = causal;
+  L.workspace = ns->scratch;
+  L.status = ns->status;
+  L.seq = next_seq();
+  L.num_sms = ns->num_sms;
+  CUtensorMap maps[6];
+  if (encode_bf16(&maps[0], q, d, N, BH) || encode_bf16(&maps[1], k, d, N, BH) ||
+      encode_bf16(&maps[2], v, d, N, BH) || encode_bf16(&maps[3], dO, d, N, BH) ||
+      encode_bf16(&maps[4], dk, d, N, BH) || encode_bf16(&maps[5], dv, d, N, BH))
+    return FA_ERR_CUDA;
+  cudaError_t e = fa::bwd_launch(L, maps, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
