@@ -66,7 +66,9 @@ struct BwdCfg {
   static constexpr int kOffL = kOffdS + 32768;  // [2][128] fp32
   static constexpr int kOffDv = kOffL + 1024;   // [2][128] fp32
   static constexpr int kOffBar = kOffDv + 1024;
-  static constexpr int kSmemBytes = kOffBar + 256;
+  static constexpr int kNumBars = 14;  // then the TMEM address slot and the abort flag
+  static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
   static constexpr int kThreads = 448;
   static constexpr uint32_t kColS = 0, kColdP = 128, kColdK = 256, kColdV = 256 + D;
   static constexpr uint32_t kColdQ = (D == 128) ? 128 : 384;
@@ -174,7 +176,7 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t *bar_dq_empty = bars + 11;
   uint64_t *bar_epi = bars + 12;
   uint64_t *bar_drain = bars + 13;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   uint8_t *sK = smem + C::kOffK;
@@ -269,13 +271,19 @@ __global__ void __launch_bounds__(448, 1)
       constexpr uint32_t id_ss = make_idesc_bf16(128, 128, 0, 0);     // S^T, dP^T
       constexpr uint32_t id_kxmn = make_idesc_bf16(128, D, 0, 1);     // dV (A in TMEM), dK
       constexpr uint32_t id_mnmn = make_idesc_bf16(128, D, 1, 1);     // dQ
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), adS = smem_u32(sdS);
+      // Base descriptors (K-major "k" and MN-major "m" views), advanced per k-step.
+      const uint64_t dKk = make_sdesc(smem_u32(sK), 16, 1024), dKm = make_sdesc(smem_u32(sK), 16384, 1024);
+      const uint64_t dVk = make_sdesc(smem_u32(sV), 16, 1024);
+      const uint64_t dSk = make_sdesc(smem_u32(sdS), 16, 1024), dSm = make_sdesc(smem_u32(sdS), 16384, 1024);
+      const uint64_t dQk0 = make_sdesc(smem_u32(sQ), 16, 1024), dQm0 = make_sdesc(smem_u32(sQ), 16384, 1024);
+      const uint64_t dOk0 = make_sdesc(smem_u32(sdO), 16, 1024), dOm0 = make_sdesc(smem_u32(sdO), 16384, 1024);
       const uint32_t tS = tmem + C::kColS, tdP = tmem + C::kColdP, tdK = tmem + C::kColdK;
       const uint32_t tdV = tmem + C::kColdV, tdQ = tmem + C::kColdQ;
       bool ok = mbar_wait(ctx, bar_kv, 0, kBTagKV);
       for (int it = 0; it < n_it && ok; ++it) {
         const int s = it & 1, n = it >> 1;
-        const uint32_t aQ = smem_u32(sQ + s * C::kTile), adO = smem_u32(sdO + s * C::kTile);
+        const uint64_t dQk = sdesc_add(dQk0, s * C::kTile), dQm = sdesc_add(dQm0, s * C::kTile);
+        const uint64_t dOk = sdesc_add(dOk0, s * C::kTile), dOm = sdesc_add(dOm0, s * C::kTile);
         ok = mbar_wait(ctx, &bar_qdo_full[s], n & 1, kBTagQdoFull);
         if (ok && it > 0) ok = mbar_wait(ctx, bar_dv_done, (it - 1) & 1, kBTagDvDone);
         if (!ok) break;
@@ -283,7 +291,7 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_ss(tS, make_sdesc(aK + off, 16, 1024), make_sdesc(aQ + off, 16, 1024), id_ss, ks > 0);
+          mma_ss(tS, sdesc_add(dKk, off), sdesc_add(dQk, off), id_ss, ks > 0);
         }
         mma_commit(bar_s_full);
         if (D == 128 && it > 0) {
@@ -294,7 +302,7 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_ss(tdP, make_sdesc(aV + off, 16, 1024), make_sdesc(adO + off, 16, 1024), id_ss, ks > 0);
+          mma_ss(tdP, sdesc_add(dVk, off), sdesc_add(dOk, off), id_ss, ks > 0);
         }
         mma_commit(bar_dp_full);
         ok = mbar_wait(ctx, bar_p_full, it & 1, kBTagPFull);
@@ -302,7 +310,7 @@ __global__ void __launch_bounds__(448, 1)
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_ts(tdV, tS + ks * 8, make_sdesc(adO + ks * 2048, 16384, 1024), id_kxmn, (it > 0 || ks > 0) ? 1u : 0u);
+          mma_ts(tdV, tS + ks * 8, sdesc_add(dOm, ks * 2048), id_kxmn, (it > 0 || ks > 0) ? 1u : 0u);
         mma_commit(bar_dv_done);
         ok = mbar_wait(ctx, bar_ds_full, it & 1, kBTagDsFull);
         if (!ok) break;
@@ -310,8 +318,7 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_ss(tdK, make_sdesc(adS + off, 16, 1024), make_sdesc(aQ + ks * 2048, 16384, 1024), id_kxmn,
-                 (it > 0 || ks > 0) ? 1u : 0u);
+          mma_ss(tdK, sdesc_add(dSk, off), sdesc_add(dQm, ks * 2048), id_kxmn, (it > 0 || ks > 0) ? 1u : 0u);
         }
         if (D == 64 && it > 0) {
           ok = mbar_wait(ctx, bar_dq_empty, (it - 1) & 1, kBTagDqEmpty);
@@ -320,8 +327,7 @@ __global__ void __launch_bounds__(448, 1)
         }
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_ss(tdQ, make_sdesc(adS + ks * 2048, 16384, 1024), make_sdesc(aK + ks * 2048, 16384, 1024), id_mnmn,
-                 ks > 0);
+          mma_ss(tdQ, sdesc_add(dSm, ks * 2048), sdesc_add(dKm, ks * 2048), id_mnmn, ks > 0);
         mma_commit(bar_dkq_done);
         mma_commit(&bar_qdo_empty[s]);
       }

@@ -4,17 +4,26 @@
 // the "tile inputs / compute locally / online normalisation / write compact
 // output" steps of the FlashAttention summary ("Architecture, step by step"),
 // with the online softmax of the review's "Tiling" section.  The N x N scores
-// live only in tensor memory (TMEM), one 128 x 128 tile at a time.
+// live only on chip, one 128 x 128 tile at a time: the fp32 S
+// and the bf16 P in tensor memory (TMEM).
 //
-// Roles (320 threads):
-//   warps 0-3  softmax for query tile 0 (thread t owns row t, TMEM lane t)
-//   warps 4-7  softmax for query tile 1
-//   warp  8    TMA producer: Q0, Q1 once, then K_j / V_j through a smem ring
-//   warp  9    MMA issuer (one thread): S_k = Q_k K_j^T and O_k += P_k V_j
+// Roles (352 threads):
+//   warps 0-7  softmax.  Warp w owns rows 32*(w%4)..+31 (its TMEM lane
+//              quarter) and the column half h = w/4 of every S tile.  All eight
+//              warps work on tile 0 of KV step j, then on tile 1, then on tile 0
+//              of step j+1 ...: while they run one tile's softmax, the tensor
+//              pipe runs the other tile's PV and next S.  The two warps that
+//              share rows exchange their half-row maxima through smem.
+//   warp  8    TMA producer: Q0, Q1 once, then K / V tiles through a smem ring.
+//   warp  9    MMA issuer for tile 0 (one thread); warp 10 for tile 1.  Two
+//              independent issuers let the pipe take whichever tile is ready.
+// A K/V ring stage is released when both issuers' MMAs that read it completed.
 //
 // TMEM columns (512 allocated): S0 [0,128), S1 [128,256), O0 [256,256+D),
-// O1 [256+D, 256+2D).  P_k (bf16, two per column) overwrites the first 64
-// columns of S_k once the softmax threads hold S_k in registers.
+// O1 [256+D, 256+2D).  The bf16 P (two per column) of column half h is written
+// over S columns [64h, 64h+32) -- inside the half its warp has already read --
+// and is the A operand of the PV MMA straight from TMEM.  So the next S of a
+// tile is issued only once that tile's PV has completed.
 //
 // Online softmax, in the log2 domain with c = scale*log2(e):
 //   m' = max(m, c*rowmax(S));  P = 2^(c*S - m');  l = 2^(m-m') l + rowsum(P);
@@ -24,6 +33,12 @@
 // The running max is only moved when it grows by more than 8 (a factor 256):
 // O and l are both kept relative to the same stale max, which is exact, and
 // P <= 256 cannot overflow fp32 or bf16.  Most tiles then skip the O rescale.
+// After the first KV step P is computed against the running max before the
+// row max of the new tile is known (the half maxima travel through smem in the
+// meantime); only a row whose max grew by more than 8 recomputes its P.
+// One pair in four of the exponentials runs on the FMA pipe (a cubic after
+// range reduction) instead of the MUFU unit, which is otherwise the bottleneck
+// (one exp per 4d FLOPs; at d = 128 the MUFU rate equals the tensor rate).
 #pragma once
 
 #include "ptx.cuh"
@@ -44,18 +59,34 @@ struct FwdParams {
 template <int D>
 struct FwdCfg {
   static constexpr int kTileBytes = 128 * D * 2;      // one 128 x D bf16 tile
-  static constexpr int kStages = (D == 128) ? 4 : 6;  // K/V ring depth
+  static constexpr int kStages = (D == 128) ? 4 : 8;  // K/V ring depth
   static constexpr int kBoxes = D / 64;               // 64-column TMA boxes per tile
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
-  static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-  static constexpr int kSmemBytes = kBarOff + 512;
-  static constexpr int kThreads = 320;
+  static constexpr int kXOff = kKVOff + kStages * kTileBytes;  // half-row maxima [2 tiles][2 halves][128]
+  static constexpr int kLOff = kXOff + 2048;                   // half-row sums [2 tiles][2 halves][2][128]
+  static constexpr int kBarOff = kLOff + 4096;
+  // mbarriers: q[2], kv_full/kv_empty[kStages], then 8 pairs; then the TMEM
+  // address slot and the abort flag.
+  static constexpr int kNumBars = 2 + 2 * kStages + 16;
+  static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16;
+  static constexpr int kThreads = 352;
+  static constexpr int kSoftmaxThreads = 256;
+  static constexpr int kProducerWarp = 8;
+  static constexpr int kIssuerWarp = 9;  // 9: tile 0 (and TMEM owner), 10: tile 1
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
 enum FwdTag : int {
-  kTagQ = 1, kTagKvFull = 2, kTagKvEmpty = 3, kTagSFull = 4, kTagPFull = 5, kTagPvDone = 6, kTagEpi = 7
+  kTagQ = 1, kTagKvFull = 2, kTagKvEmpty = 3, kTagSFull = 4, kTagPFull = 5, kTagPvDone = 6, kTagEpi = 7,
+  kTagXmax = 8, kTagLsum = 9
 };
+
+// Load order of the K/V ring: K tiles run one KV step ahead of V tiles
+// (K0, K1, V0, K2, V1, ..., K_{n-1}, V_{n-2}, V_{n-1}), because S of step j+1
+// is issued while P of step j is still being computed.  Ring slot of each load:
+__device__ __forceinline__ int kv_idx_k(int j) { return j == 0 ? 0 : 2 * j - 1; }
+__device__ __forceinline__ int kv_idx_v(int j, int n) { return (j + 1 < n) ? 2 * j + 2 : 2 * j + 1; }
 
 // Position of 16-byte chunk `chunk` (0..7) of row `row` in a 128-byte-swizzled
 // tile: TMA's SWIZZLE_128B pattern XORs the chunk index with row % 8.
@@ -64,7 +95,7 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
 }
 
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const FwdParams p) {
@@ -75,12 +106,15 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t *bar_q = bars + 0;                        // [2]
   uint64_t *bar_kv_full = bars + 2;                  // [kStages]
   uint64_t *bar_kv_empty = bars + 2 + C::kStages;    // [kStages]
-  uint64_t *bar_s_full = bars + 2 + 2 * C::kStages;  // [2]
-  uint64_t *bar_p_full = bar_s_full + 2;             // [2]
-  uint64_t *bar_pv_done = bar_p_full + 2;            // [2]
+  uint64_t *bar_s_full = bars + 2 + 2 * C::kStages;  // [2] S_k in TMEM
+  uint64_t *bar_p_full = bar_s_full + 2;             // [2] P_k in TMEM (and O_k rescaled)
+  uint64_t *bar_pv_done = bar_p_full + 2;            // [2] PV_k completed
   uint64_t *bar_epi = bar_pv_done + 2;               // [2]
-  uint64_t *bar_drain = bar_epi + 2;                 // [1]
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_drain + 1);
+  uint64_t *bar_drain = bar_epi + 2;                 // [2]
+  uint64_t *bar_x = bar_drain + 2;                   // [2] half-row max exchange
+  uint64_t *bar_l = bar_x + 2;                       // [2] half-row sum exchange
+  static_assert(2 + 2 * C::kStages + 16 == C::kNumBars, "barrier count");
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_l + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -111,19 +145,21 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(&bar_q[1], 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&bar_kv_full[s], 1);
-      mbar_init(&bar_kv_empty[s], 1);
+      mbar_init(&bar_kv_empty[s], 2);  // one arrival per MMA issuer
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(&bar_s_full[k], 1);
-      mbar_init(&bar_p_full[k], 128);
+      mbar_init(&bar_p_full[k], C::kSoftmaxThreads);
       mbar_init(&bar_pv_done[k], 1);
-      mbar_init(&bar_epi[k], 128);
+      mbar_init(&bar_epi[k], C::kSoftmaxThreads);
+      mbar_init(&bar_x[k], C::kSoftmaxThreads);
+      mbar_init(&bar_l[k], C::kSoftmaxThreads);
+      mbar_init(&bar_drain[k], 1);
     }
-    mbar_init(bar_drain, 1);
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == 9) {
+  if (warp == C::kIssuerWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -131,11 +167,12 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) FA_TRACE(0);
 
   uint8_t *sQ = smem + C::kQOff;
   uint8_t *sKV = smem + C::kKVOff;
 
-  if (warp == 8) {
+  if (warp == C::kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && !*abort_flag) {
       tma_prefetch_desc(&tmQ);
@@ -147,20 +184,20 @@ __global__ void __launch_bounds__(320, 1)
         tma_load_3d(&tmQ, &bar_q[0], sQ + b * 16384, b * 64, (2 * u) * 128, bh);
       int idx = 0;
       bool ok = true;
-      for (int j = 0; j < n_kv && ok; ++j) {
-        for (int t = 0; t < 2 && ok; ++t) {
-          const int s = idx % C::kStages, n = idx / C::kStages;
-          if (n > 0 && !mbar_wait(ctx, &bar_kv_empty[s], (n - 1) & 1, kTagKvEmpty)) { ok = false; break; }
-          uint8_t *dst = sKV + s * C::kTileBytes;
-          mbar_arrive_expect_tx(&bar_kv_full[s], C::kTileBytes);
+      for (; idx < 2 * n_kv && ok; ++idx) {
+        // Which tile is load number idx in the K-ahead order.
+        const bool is_k = (idx == 0) || ((idx & 1) && (idx + 1) / 2 < n_kv);
+        const int j = (idx == 0) ? 0 : (is_k ? (idx + 1) / 2 : (idx == 2 * n_kv - 1 ? n_kv - 1 : idx / 2 - 1));
+        const int s = idx % C::kStages, n = idx / C::kStages;
+        if (n > 0 && !mbar_wait(ctx, &bar_kv_empty[s], (n - 1) & 1, kTagKvEmpty)) { ok = false; break; }
+        uint8_t *dst = sKV + s * C::kTileBytes;
+        mbar_arrive_expect_tx(&bar_kv_full[s], C::kTileBytes);
+        for (int b = 0; b < C::kBoxes; ++b)
+          tma_load_3d(is_k ? &tmK : &tmV, &bar_kv_full[s], dst + b * 16384, b * 64, j * 128, bh);
+        if (idx == 0) {
+          mbar_arrive_expect_tx(&bar_q[1], C::kTileBytes);
           for (int b = 0; b < C::kBoxes; ++b)
-            tma_load_3d(t == 0 ? &tmK : &tmV, &bar_kv_full[s], dst + b * 16384, b * 64, j * 128, bh);
-          ++idx;
-          if (j == 0 && t == 0) {
-            mbar_arrive_expect_tx(&bar_q[1], C::kTileBytes);
-            for (int b = 0; b < C::kBoxes; ++b)
-              tma_load_3d(&tmQ, &bar_q[1], sQ + C::kTileBytes + b * 16384, b * 64, (2 * u + 1) * 128, bh);
-          }
+            tma_load_3d(&tmQ, &bar_q[1], sQ + C::kTileBytes + b * 16384, b * 64, (2 * u + 1) * 128, bh);
         }
       }
       if (!ok) {
@@ -174,157 +211,207 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == C::kIssuerWarp || warp == C::kIssuerWarp + 1) {
+    // ------------------------------------------------------------ MMA issuers
+    const int k = warp - C::kIssuerWarp;  // query tile owned by this issuer
     if (lane == 0 && !*abort_flag) {
       constexpr uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = make_idesc_bf16(128, D, 0, 1);
-      const uint32_t q_addr[2] = {smem_u32(sQ), smem_u32(sQ + C::kTileBytes)};
-      const uint32_t kv_addr = smem_u32(sKV);
-      const uint32_t tS[2] = {tmem, tmem + 128};
-      const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
-      bool ok = mbar_wait(ctx, &bar_q[0], 0, kTagQ);
+      // Base descriptors: Q_k (K-major), ring stage 0 as K (K-major) and as V (MN-major).
+      const uint64_t q_desc = make_sdesc(smem_u32(sQ + k * C::kTileBytes), 16, 1024);
+      const uint64_t k_desc0 = make_sdesc(smem_u32(sKV), 16, 1024);
+      const uint64_t v_desc0 = make_sdesc(smem_u32(sKV), 16384, 1024);
+      const uint32_t tS = tmem + 128 * k;
+      const uint32_t tO = tmem + 256 + k * D;
+      const int n_k = (k == 0) ? n_kv0 : n_kv1;
+      bool ok = mbar_wait(ctx, &bar_q[k], 0, kTagQ);
       for (int j = 0; j < n_kv && ok; ++j) {
-        const int iK = 2 * j, iV = 2 * j + 1;
-        const int sK = iK % C::kStages, sV = iV % C::kStages;
+        const int iK = kv_idx_k(j), sK = iK % C::kStages;
+        const int iV = kv_idx_v(j, n_kv), sV = iV % C::kStages;
+        // Arrivals on kv_empty must follow the matching kv_full phase, so even
+        // a tile that skips K_j / V_j (causal tile 0 past its diagonal) waits.
         ok = mbar_wait(ctx, &bar_kv_full[sK], (iK / C::kStages) & 1, kTagKvFull);
         if (!ok) break;
-        tc_fence_after();
-        const uint32_t k_addr = kv_addr + sK * C::kTileBytes;
-        for (int k = 0; k < 2 && ok; ++k) {
-          if (k == 0 && j >= n_kv0) continue;
-          if (k == 1 && j == 0) ok = mbar_wait(ctx, &bar_q[1], 0, kTagQ);
-          // S_k is free once PV_k of the previous tile has consumed P_k.
-          if (ok && j > 0) ok = mbar_wait(ctx, &bar_pv_done[k], (j - 1) & 1, kTagPvDone);
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-            mma_ss(tS[k], make_sdesc(q_addr[k] + off, 16, 1024), make_sdesc(k_addr + off, 16, 1024), idesc_qk,
-                   ks > 0);
-          }
-          mma_commit(&bar_s_full[k]);
+        if (j >= n_k) {
+          mbar_arrive(&bar_kv_empty[sK]);
+          ok = mbar_wait(ctx, &bar_kv_full[sV], (iV / C::kStages) & 1, kTagKvFull);
+          if (ok) mbar_arrive(&bar_kv_empty[sV]);
+          continue;
         }
+        // S_k aliases P_k: the previous PV_k must have consumed P_k.
+        if (j > 0) ok = mbar_wait(ctx, &bar_pv_done[k], (j - 1) & 1, kTagPvDone);
         if (!ok) break;
+        tc_fence_after();
+        const uint64_t k_desc = sdesc_add(k_desc0, sK * C::kTileBytes);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          mma_ss(tS, sdesc_add(q_desc, off), sdesc_add(k_desc, off), idesc_qk, ks > 0);
+        }
+        mma_commit(&bar_s_full[k]);
         mma_commit(&bar_kv_empty[sK]);
+        FA_TRACE(16 + k * 256 + 4 * j + 0);
         ok = mbar_wait(ctx, &bar_kv_full[sV], (iV / C::kStages) & 1, kTagKvFull);
+        if (ok) ok = mbar_wait(ctx, &bar_p_full[k], j & 1, kTagPFull);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t v_addr = kv_addr + sV * C::kTileBytes;
-        for (int k = 0; k < 2 && ok; ++k) {
-          if (k == 0 && j >= n_kv0) continue;
-          ok = mbar_wait(ctx, &bar_p_full[k], j & 1, kTagPFull);
-          if (!ok) break;
-          tc_fence_after();
+        FA_TRACE(16 + k * 256 + 4 * j + 2);
+        const uint64_t v_desc = sdesc_add(v_desc0, sV * C::kTileBytes);
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            mma_ts(tO[k], tS[k] + ks * 8, make_sdesc(v_addr + ks * 2048, 16384, 1024), idesc_pv,
-                   (j > 0 || ks > 0) ? 1u : 0u);
-          }
-          mma_commit(&bar_pv_done[k]);
-        }
-        if (!ok) break;
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ts(tO, tS + ks * 8 + (ks >= 4 ? 32 : 0), sdesc_add(v_desc, ks * 2048), idesc_pv,
+                 (j > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(&bar_pv_done[k]);
         mma_commit(&bar_kv_empty[sV]);
+        FA_TRACE(16 + k * 256 + 4 * j + 1);
       }
       if (!ok) {
-        // Let every MMA already issued finish before TMEM is released.
-        mma_commit(bar_drain);
-        mbar_drain(bar_drain, 0);
+        // Let every MMA this thread issued finish before TMEM is released.
+        mma_commit(&bar_drain[k]);
+        mbar_drain(&bar_drain[k], 0);
       }
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
-    const int k = warp >> 2;  // query tile handled by this warpgroup
-    const int r = (warp & 3) * 32 + lane;  // row within the tile == TMEM lane
-    const int qt = 2 * u + k;              // query tile index
-    const int n_k = (k == 0) ? n_kv0 : n_kv1;
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_off + 128 * k;
-    const uint32_t tO = tmem + lane_off + 256 + k * D;
+    const int h = warp >> 2;                 // column half of every S tile
+    const int rq = warp & 3;                 // TMEM lane quarter
+    const int r = rq * 32 + lane;            // row within the tile == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(rq * 32) << 16;
+    float *xm = reinterpret_cast<float *>(smem + C::kXOff);  // [k][h][128]
     const float c = p.scale_log2;
-    float m = -INFINITY, l = 0.f, lr = 0.f;  // running max, row sum, rounded row sum
+    const uint64_t c2 = f2pack(c, c);
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, lr[2] = {0.f, 0.f};
+    const int n_k[2] = {n_kv0, n_kv1};
     bool ok = !*abort_flag;
-    for (int j = 0; j < n_k && ok; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_s_full[k], j & 1, kTagSFull));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t s[128];
-      tmem_ld32(tS + 0, s + 0);
-      tmem_ld32(tS + 32, s + 32);
-      tmem_ld32(tS + 64, s + 64);
-      tmem_ld32(tS + 96, s + 96);
-      tmem_wait_ld();
-      // Keys j*128 + col are valid when col < nvalid (tail of N, causal diagonal).
-      int nvalid = min(128, p.N - j * 128);
-      if (CAUSAL && j == qt) nvalid = min(nvalid, r + 1);
-      if (nvalid < 128) {
-#pragma unroll
-        for (int cc = 0; cc < 128; ++cc)
-          if (cc >= nvalid) s[cc] = __float_as_uint(-INFINITY);
-      }
-      float mx = __uint_as_float(s[0]);
-#pragma unroll
-      for (int cc = 1; cc < 128; ++cc) mx = fmaxf(mx, __uint_as_float(s[cc]));
-      const float m_cand = mx * c;
-      float alpha = 1.f;
-      bool rescale = false;
-      if (m_cand > m + 8.f) {  // also taken on the first tile (m = -inf)
-        alpha = ex2(m - m_cand);
-        rescale = (j > 0);
-        m = m_cand;
-      }
-      const float neg = (m == -INFINITY) ? 0.f : -m;
-      // Two row sums: of P in fp32 (for the LSE) and of P as rounded to bf16,
-      // i.e. exactly the weights the PV MMA multiplies V with (for O's
-      // normaliser, so that O is a convex combination of the rows of V).
-      float sum0 = 0.f, sum1 = 0.f, rsum0 = 0.f, rsum1 = 0.f;
-      uint32_t pk[64];
-#pragma unroll
-      for (int cc = 0; cc < 64; ++cc) {
-        const float a = ex2(fmaf(__uint_as_float(s[2 * cc]), c, neg));
-        const float b = ex2(fmaf(__uint_as_float(s[2 * cc + 1]), c, neg));
-        sum0 += a;
-        sum1 += b;
-        pk[cc] = pack_bf16(a, b);
-        rsum0 += __uint_as_float(pk[cc] << 16);
-        rsum1 += __uint_as_float(pk[cc] & 0xFFFF0000u);
-      }
-      l = l * alpha + (sum0 + sum1);
-      lr = lr * alpha + (rsum0 + rsum1);
-      if (__any_sync(0xffffffffu, rescale)) {
-        // O_k still holds the previous tile's PV: wait for it, then rescale.
-        ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_pv_done[k], (j - 1) & 1, kTagPvDone));
+    for (int j = 0; j < n_kv && ok; ++j) {
+      for (int k = 0; k < 2 && ok; ++k) {
+        if (j >= n_k[k]) continue;
+        const int qt = 2 * u + k;
+        const uint32_t tS = tmem + lane_off + 128 * k + 64 * h;
+        ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_s_full[k], j & 1, kTagSFull));
         if (!ok) break;
         tc_fence_after();
+        if (r == 0 && h == 0) FA_TRACE(528 + k * 256 + 4 * j + 0);
+        uint32_t s[64];
+        tmem_ld32(tS, s);
+        tmem_ld32(tS + 32, s + 32);
+        tmem_wait_ld();
+        // Keys j*128 + 64h + col are valid when col < nv (tail of N, causal diagonal).
+        int nvalid = min(128, p.N - j * 128);
+        if (CAUSAL && j == qt) nvalid = min(nvalid, r + 1);
+        const int nv = nvalid - 64 * h;
+        if (nv < 64) {
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t o[32];
-          tmem_ld32(tO + ch * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
-          tmem_st32(tO + ch * 32, o);
+          for (int cc = 0; cc < 64; ++cc)
+            if (cc >= nv) s[cc] = __float_as_uint(-INFINITY);
         }
+        float ma = __uint_as_float(s[0]), mb = __uint_as_float(s[32]);
+#pragma unroll
+        for (int t = 1; t < 31; t += 2) {
+          ma = fmax3(ma, __uint_as_float(s[t]), __uint_as_float(s[t + 1]));
+          mb = fmax3(mb, __uint_as_float(s[32 + t]), __uint_as_float(s[33 + t]));
+        }
+        const float mh = fmax3(ma, mb, fmaxf(__uint_as_float(s[31]), __uint_as_float(s[63])));
+        xm[(k * 2 + h) * 128 + r] = mh;
+        mbar_arrive(&bar_x[k]);
+        // P = 2^(c*S - m) for this half row, with the row sums of P in fp32
+        // (for the LSE) and of P rounded to bf16 (the PV weights; O's normaliser).
+        uint32_t pk[32];
+        float psum = 0.f, prsum = 0.f;
+        auto exps = [&](float mref) {
+          const float neg = (mref == -INFINITY) ? 0.f : -mref;
+          const uint64_t n2 = f2pack(neg, neg);
+          uint64_t acc[2] = {0ull, 0ull}, racc[2] = {0ull, 0ull};
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) {
+            const uint64_t x2 = ffma2(f2pack(__uint_as_float(s[2 * cc]), __uint_as_float(s[2 * cc + 1])), c2, n2);
+            float x0, x1, a, b;
+            f2unpack(x2, x0, x1);
+            if ((cc & 3) == 3) {
+              exp2_poly_pair(x0, x1, a, b);
+            } else {
+              a = ex2(x0);
+              b = ex2(x1);
+            }
+            acc[cc & 1] = fadd2(acc[cc & 1], f2pack(a, b));
+            pk[cc] = pack_bf16(a, b);
+            racc[cc & 1] =
+                fadd2(racc[cc & 1], f2pack(__uint_as_float(pk[cc] << 16), __uint_as_float(pk[cc] & 0xFFFF0000u)));
+          }
+          float u0, u1, u2, u3, v0, v1, v2, v3;
+          f2unpack(acc[0], u0, u1);
+          f2unpack(acc[1], u2, u3);
+          f2unpack(racc[0], v0, v1);
+          f2unpack(racc[1], v2, v3);
+          psum = (u0 + u1) + (u2 + u3);
+          prsum = (v0 + v1) + (v2 + v3);
+        };
+        const float m_old = m[k];
+        if (m_old != -INFINITY) exps(m_old);  // optimistic: the running max usually holds
+        ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_x[k], j & 1, kTagXmax));
+        if (!ok) break;
+        const float m_cand = fmaxf(mh, xm[(k * 2 + (h ^ 1)) * 128 + r]) * c;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (m_cand > m_old + 8.f) {  // also taken on the first tile (m = -inf)
+          alpha = ex2(m_old - m_cand);
+          rescale = (m_old != -INFINITY);
+          m[k] = m_cand;
+          exps(m_cand);
+        }
+        l[k] = l[k] * alpha + psum;
+        lr[k] = lr[k] * alpha + prsum;
+        if (__any_sync(0xffffffffu, rescale)) {
+          // O_k still holds the previous step's PV: wait for it, then rescale
+          // this warp's column half of O.
+          ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_pv_done[k], (j - 1) & 1, kTagPvDone));
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t tO = tmem + lane_off + 256 + k * D + h * (D / 2);
+#pragma unroll
+          for (int ch = 0; ch < D / 64; ++ch) {
+            uint32_t o[32];
+            tmem_ld32(tO + ch * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
+            tmem_st32(tO + ch * 32, o);
+          }
+        }
+        tmem_st32(tS, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar_p_full[k]);
+        if (r == 0 && h == 0) FA_TRACE(528 + k * 256 + 4 * j + 1);
+        if (lane == 0 && j < 16) FA_TRACE(1024 + (k * 8 + warp) * 16 + j);
       }
-      tmem_st32(tS + 0, pk + 0);
-      tmem_st32(tS + 32, pk + 32);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bar_p_full[k]);
     }
     // ---------------------------------------------------------- epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_pv_done[k], (n_k - 1) & 1, kTagPvDone));
-    if (ok) {
+    for (int k = 0; k < 2 && ok; ++k) {
+      const int qt = 2 * u + k;
+      ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_pv_done[k], (n_k[k] - 1) & 1, kTagPvDone));
+      if (!ok) break;
       tc_fence_after();
-      const float inv_l = 1.f / lr;
+      // Whole-row sums from the two column halves.
+      float *ls = reinterpret_cast<float *>(smem + C::kLOff) + k * 512;  // [h][2][128]
+      ls[(h * 2 + 0) * 128 + r] = l[k];
+      ls[(h * 2 + 1) * 128 + r] = lr[k];
+      mbar_arrive(&bar_l[k]);
+      ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_l[k], 0, kTagLsum));
+      if (!ok) break;
+      if (r == 0 && h == 0) FA_TRACE(4 + k);
+      const float lt = l[k] + ls[((h ^ 1) * 2 + 0) * 128 + r];
+      const float lrt = lr[k] + ls[((h ^ 1) * 2 + 1) * 128 + r];
+      const float inv_l = 1.f / lrt;
       uint8_t *stage = sQ + k * C::kTileBytes;  // Q_k is dead: all its MMAs completed
       const uint32_t stage_addr = smem_u32(stage);
+      const uint32_t tO = tmem + lane_off + 256 + k * D;
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
+      for (int ch = 0; ch < D / 64; ++ch) {
+        const int col0 = h * (D / 2) + 32 * ch;  // first feature of this 32-column chunk
         uint32_t o[32];
-        tmem_ld32(tO + ch * 32, o);
+        tmem_ld32(tO + col0, o);
         tmem_wait_ld();
         uint32_t w[16];
 #pragma unroll
@@ -339,29 +426,27 @@ __global__ void __launch_bounds__(320, 1)
             const float a = __uint_as_float(o[2 * t]) * inv_l, b = __uint_as_float(o[2 * t + 1]) * inv_l;
             lo[t] = pack_bf16(a - __uint_as_float(w[t] << 16), b - __uint_as_float(w[t] & 0xFFFF0000u));
           }
-          uint4 *dst = reinterpret_cast<uint4 *>(p.o_lo + (static_cast<size_t>(bh) * p.N + qt * 128 + r) * D +
-                                                 ch * 32);
+          uint4 *dst = reinterpret_cast<uint4 *>(p.o_lo + (static_cast<size_t>(bh) * p.N + qt * 128 + r) * D + col0);
 #pragma unroll
           for (int t = 0; t < 4; ++t) dst[t] = make_uint4(lo[4 * t], lo[4 * t + 1], lo[4 * t + 2], lo[4 * t + 3]);
         }
-        const int box = ch >> 1;
+        const int box = col0 >> 6, chunk0 = (col0 & 63) >> 3;
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int chunk = (ch & 1) * 4 + t;
-          st_shared_v4(stage_addr + box * 16384 + sw128_offset(r, chunk), w[4 * t], w[4 * t + 1], w[4 * t + 2],
-                       w[4 * t + 3]);
-        }
+        for (int t = 0; t < 4; ++t)
+          st_shared_v4(stage_addr + box * 16384 + sw128_offset(r, chunk0 + t), w[4 * t], w[4 * t + 1],
+                       w[4 * t + 2], w[4 * t + 3]);
       }
       const int grow = qt * 128 + r;
-      if (grow < p.N) p.lse[static_cast<size_t>(bh) * p.N + grow] = (m + log2f(l)) * 0.69314718055994531f;
-      // Make the generic-proxy smem writes visible to TMA, then one thread of
-      // the warpgroup stores the tile once all 128 rows have arrived.
+      if (h == 0 && grow < p.N) p.lse[static_cast<size_t>(bh) * p.N + grow] = (m[k] + log2f(lt)) * 0.69314718055994531f;
+      // Make the generic-proxy smem writes visible to TMA, then one thread
+      // stores the tile once all softmax threads have written their part.
       fence_proxy_async_smem();
       mbar_arrive(&bar_epi[k]);
-      if (r == 0 && mbar_wait(ctx, &bar_epi[k], 0, kTagEpi) && qt * 128 < p.N) {
+      if (warp == 0 && lane == 0 && mbar_wait(ctx, &bar_epi[k], 0, kTagEpi) && qt * 128 < p.N) {
         for (int b = 0; b < C::kBoxes; ++b) tma_store_3d(&tmO, stage + b * 16384, b * 64, qt * 128, bh);
         bulk_commit();
         bulk_wait_read<0>();
+        FA_TRACE(6 + k);
       }
     }
     __syncwarp();
@@ -370,7 +455,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 9) tmem_dealloc(tmem, 512);
+  if (warp == C::kIssuerWarp) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace fa

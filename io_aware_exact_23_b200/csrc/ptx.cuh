@@ -7,6 +7,12 @@
 #include <cstdint>
 #include <cuda.h>
 
+// Pipeline event hook: a no-op in library builds.  A profiling build may define
+// FA_TRACE(slot) before including this header to timestamp pipeline events.
+#ifndef FA_TRACE
+#define FA_TRACE(slot) ((void)0)
+#endif
+
 namespace fa {
 
 // ----------------------------------------------------------- status word
@@ -201,6 +207,16 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo_byte
   return d;
 }
 
+// A descriptor moved by `bytes` (a multiple of 16): only the start-address
+// field (bits 0..13, address >> 4) changes, and it cannot carry into the next
+// field because every shared-memory address is below 256 KB.  Issuing threads
+// build one base descriptor per buffer up front and advance it with this single
+// add, so the MMA issue loop stays short (the MMA pipe drains a 128x128x16
+// instruction in about 64 cycles; a slower issue loop starves it).
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) {
+  return desc + static_cast<uint64_t>(bytes >> 4);
+}
+
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B,
 // A/B major-ness (0 = K-major, 1 = MN-major), N >> 3 at bit 17, M >> 4 at bit 24.
 __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
@@ -287,6 +303,60 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction, two lanes of work).
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Software 2^x for a pair, on the FMA pipe (relieves the MUFU unit):
+// 2^x = 2^n * p(f) with n = rint(x), f = x - n in [-1/2, 1/2] and p the cubic
+// minimax fit of 2^f on that interval (relative error 7.5e-5; coefficients from
+// csrc/gen_exp2_poly.py, a Remez fit of our own).  n is read from the low bits
+// of x + 1.5*2^23 and added to p's exponent field.  Inputs are clamped at -126
+// (so n >= -126 and the exponent field stays >= 0: masked -inf entries give a
+// positive value below 2^-125 instead of 0).  Inputs above 127 are not expected.
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float &y0, float &y1) {
+  const uint64_t kMagic = f2pack(12582912.f, 12582912.f);
+  const uint64_t kNegMagic = f2pack(-12582912.f, -12582912.f);
+  const uint64_t kNegOne = f2pack(-1.f, -1.f);
+  const uint64_t c0 = f2pack(0.9999280571937561f, 0.9999280571937561f);
+  const uint64_t c1 = f2pack(0.6932609677314758f, 0.6932609677314758f);
+  const uint64_t c2 = f2pack(0.2426111251115799f, 0.2426111251115799f);
+  const uint64_t c3 = f2pack(0.0551716685295105f, 0.0551716685295105f);
+  const uint64_t x = f2pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = fadd2(x, kMagic);          // rint(x) in the low mantissa bits
+  const uint64_t r = fadd2(t, kNegMagic);       // rint(x) as a float
+  const uint64_t f = ffma2(r, kNegOne, x);      // x - rint(x), exact
+  uint64_t pp = ffma2(f, c3, c2);
+  pp = ffma2(pp, f, c1);
+  pp = ffma2(pp, f, c0);
+  float p0, p1, t0, t1;
+  f2unpack(pp, p0, p1);
+  f2unpack(t, t0, t1);
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` lands in bits 0..15.
