@@ -253,10 +253,11 @@ int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o, const 
   L.seq = next_seq();
   L.num_sms = ds->num_sms;
   L.events = reinterpret_cast<cudaEvent_t const *>(events);
-  CUtensorMap maps[6];
+  CUtensorMap maps[7];
   if (encode_bf16(&maps[0], q, d, N, BH) || encode_bf16(&maps[1], k, d, N, BH) ||
       encode_bf16(&maps[2], v, d, N, BH) || encode_bf16(&maps[3], dO, d, N, BH) ||
-      encode_bf16(&maps[4], dk, d, N, BH) || encode_bf16(&maps[5], dv, d, N, BH))
+      encode_bf16(&maps[4], dk, d, N, BH) || encode_bf16(&maps[5], dv, d, N, BH) ||
+      encode_3d(&maps[6], L.workspace, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, BH, 32))
     return FA_ERR_CUDA;
   cudaError_t e = fa::bwd_launch(L, maps, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -384,10 +385,11 @@ extern "C" int fa_bwd_noalloc(const void *q, const void *k, const void *v, const
   L.status = ns->status;
   L.seq = next_seq();
   L.num_sms = ns->num_sms;
-  CUtensorMap maps[6];
+  CUtensorMap maps[7];
   if (encode_bf16(&maps[0], q, d, N, BH) || encode_bf16(&maps[1], k, d, N, BH) ||
       encode_bf16(&maps[2], v, d, N, BH) || encode_bf16(&maps[3], dO, d, N, BH) ||
-      encode_bf16(&maps[4], dk, d, N, BH) || encode_bf16(&maps[5], dv, d, N, BH))
+      encode_bf16(&maps[4], dk, d, N, BH) || encode_bf16(&maps[5], dv, d, N, BH) ||
+      encode_3d(&maps[6], L.workspace, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, BH, 32))
     return FA_ERR_CUDA;
   cudaError_t e = fa::bwd_launch(L, maps, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;

@@ -21,7 +21,11 @@
 // fa_bwd_kernel roles (448 threads):
 //   warps 0-3   compute, query columns 0..63 of each tile (thread = key row)
 //   warps 4-7   compute, query columns 64..127
-//   warps 8-11  dQ drain: TMEM dQ rows -> fp32 adds into the accumulator
+//   warps 8-11  dQ drain: TMEM dQ rows -> registers (TMEM released at once) ->
+//               scale -> the Q_i / dO_i stage buffers of the finished tile
+//               (together exactly one fp32 dQ tile) -> TMA bulk reduce-add into
+//               the fp32 accumulator in L2; the drain then hands the stage back
+//               to the producer
 //   warp  12    TMA producer: K_j, V_j once; Q_i, dO_i, LSE_i, D_i per tile (2 stages)
 //   warp  13    MMA issuer (one thread), five MMAs per query tile:
 //                 S^T  = K_j Q_i^T      (smem x smem)      -> TMEM
@@ -35,6 +39,9 @@
 // when D = 128 (dP^T is dead once dS is formed) and [384,448) when D = 64.
 // dS^T (bf16) is written to smem in the 128-byte-swizzled K-major layout,
 // which is at the same time the MN-major layout of dS for the dQ MMA.
+// CTAs are ordered in chunks of kHeadChunk heads, heaviest key tiles first
+// within a chunk: the fp32 dQ rows of a chunk stay resident in L2 while its
+// key tiles add into them.
 #pragma once
 
 #include "ptx.cuh"
@@ -54,6 +61,18 @@ struct BwdParams {
   float scale;
 };
 
+constexpr int kHeadChunk = 8;  // heads whose CTAs are scheduled together
+
+// CTA -> (head, key tile): chunks of kHeadChunk heads; inside a chunk all heads'
+// key tile 0 first, then tile 1, ... (tile 0 is the heaviest when causal).
+__device__ __forceinline__ void bwd_unit(int block, int BH, int nkv, int &bh, int &j) {
+  const int per_chunk = kHeadChunk * nkv;
+  const int c = block / per_chunk, rem = block % per_chunk;
+  const int g = min(kHeadChunk, BH - c * kHeadChunk);
+  j = rem / g;
+  bh = c * kHeadChunk + rem % g;
+}
+
 template <int D>
 struct BwdCfg {
   static constexpr int kTile = 128 * D * 2;
@@ -66,7 +85,7 @@ struct BwdCfg {
   static constexpr int kOffL = kOffdS + 32768;  // [2][128] fp32
   static constexpr int kOffDv = kOffL + 1024;   // [2][128] fp32
   static constexpr int kOffBar = kOffDv + 1024;
-  static constexpr int kNumBars = 14;  // then the TMEM address slot and the abort flag
+  static constexpr int kNumBars = 17;  // then the TMEM address slot and the abort flag
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static constexpr int kThreads = 448;
@@ -76,7 +95,8 @@ struct BwdCfg {
 
 enum BwdTag : int {
   kBTagKV = 11, kBTagQdoFull = 12, kBTagQdoEmpty = 13, kBTagSFull = 14, kBTagDpFull = 15, kBTagPFull = 16,
-  kBTagDsFull = 17, kBTagDvDone = 18, kBTagDkqDone = 19, kBTagDqEmpty = 20, kBTagEpi = 21
+  kBTagDsFull = 17, kBTagDvDone = 18, kBTagDkqDone = 19, kBTagDqEmpty = 20, kBTagEpi = 21, kBTagDrained = 22,
+  kBTagStage = 23
 };
 
 __device__ __forceinline__ uint32_t bsw128(int row, int chunk) {
@@ -159,7 +179,7 @@ __global__ void __launch_bounds__(448, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                   const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmdQacc, const BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
 
@@ -176,6 +196,9 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t *bar_dq_empty = bars + 11;
   uint64_t *bar_epi = bars + 12;
   uint64_t *bar_drain = bars + 13;
+  uint64_t *bar_drained = bars + 14;   // the dQ drain has finished with every stage buffer
+  uint64_t *bar_stage = bars + 15;     // dQ drain: all 128 rows staged
+  uint64_t *bar_unused = bars + 16;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -189,9 +212,9 @@ __global__ void __launch_bounds__(448, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x % p.BH;
-  const int j = blockIdx.x / p.BH;  // key tile; small j first (longest first when causal)
   const int nq = (p.N + 127) / 128;
+  int bh, j;  // head and key tile of this CTA
+  bwd_unit(blockIdx.x, p.BH, nq, bh, j);
   const int i0 = CAUSAL ? j : 0;
   const int n_it = nq - i0;
 
@@ -214,6 +237,9 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(bar_dq_empty, 128);
     mbar_init(bar_epi, 256);
     mbar_init(bar_drain, 1);
+    mbar_init(bar_drained, 1);
+    mbar_init(bar_stage, 128);
+    mbar_init(bar_unused, 1);
     fence_barrier_init();
     fence_proxy_async_smem();
   }
@@ -225,6 +251,7 @@ __global__ void __launch_bounds__(448, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) FA_TRACE(0);
 
   if (warp == 12) {
     // ------------------------------------------------------------ producer
@@ -294,6 +321,7 @@ __global__ void __launch_bounds__(448, 1)
           mma_ss(tS, sdesc_add(dKk, off), sdesc_add(dQk, off), id_ss, ks > 0);
         }
         mma_commit(bar_s_full);
+        FA_TRACE(16 + it * 8 + 0);
         if (D == 128 && it > 0) {
           ok = mbar_wait(ctx, bar_dq_empty, (it - 1) & 1, kBTagDqEmpty);
           if (!ok) break;
@@ -305,6 +333,7 @@ __global__ void __launch_bounds__(448, 1)
           mma_ss(tdP, sdesc_add(dVk, off), sdesc_add(dOk, off), id_ss, ks > 0);
         }
         mma_commit(bar_dp_full);
+        FA_TRACE(16 + it * 8 + 1);
         ok = mbar_wait(ctx, bar_p_full, it & 1, kBTagPFull);
         if (!ok) break;
         tc_fence_after();
@@ -312,6 +341,7 @@ __global__ void __launch_bounds__(448, 1)
         for (int ks = 0; ks < 8; ++ks)
           mma_ts(tdV, tS + ks * 8, sdesc_add(dOm, ks * 2048), id_kxmn, (it > 0 || ks > 0) ? 1u : 0u);
         mma_commit(bar_dv_done);
+        FA_TRACE(16 + it * 8 + 2);
         ok = mbar_wait(ctx, bar_ds_full, it & 1, kBTagDsFull);
         if (!ok) break;
         tc_fence_after();
@@ -328,8 +358,8 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           mma_ss(tdQ, sdesc_add(dSm, ks * 2048), sdesc_add(dKm, ks * 2048), id_mnmn, ks > 0);
-        mma_commit(bar_dkq_done);
-        mma_commit(&bar_qdo_empty[s]);
+        mma_commit(bar_dkq_done);  // the dQ drain releases the Q/dO stage after staging through it
+        FA_TRACE(16 + it * 8 + 3);
       }
       if (!ok) {
         mma_commit(bar_drain);
@@ -354,6 +384,7 @@ __global__ void __launch_bounds__(448, 1)
                                        mbar_wait(ctx, &bar_qdo_full[s], n & 1, kBTagQdoFull));
       if (!ok) break;
       tc_fence_after();
+      if (threadIdx.x == 0) FA_TRACE(16 + it * 8 + 4);
       uint32_t sv[64];
       tmem_ld32(tS + 64 * w, sv);
       tmem_ld32(tS + 64 * w + 32, sv + 32);
@@ -375,12 +406,14 @@ __global__ void __launch_bounds__(448, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p_full);
+      if (threadIdx.x == 0) FA_TRACE(16 + it * 8 + 5);
 
       ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dp_full, it & 1, kBTagDpFull));
       // The previous tile's dK / dQ MMAs read dS from smem: wait until they are done.
       if (ok && it > 0) ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, (it - 1) & 1, kBTagDkqDone));
       if (!ok) break;
       tc_fence_after();
+      if (threadIdx.x == 0) FA_TRACE(16 + it * 8 + 6);
       const float *Dv = sDv + s * 128 + 64 * w;
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
@@ -402,13 +435,16 @@ __global__ void __launch_bounds__(448, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar_ds_full);
+      if (threadIdx.x == 0) FA_TRACE(16 + it * 8 + 7);
     }
     // ---------------------------------------------------------- epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, (n_it - 1) & 1, kBTagDkqDone));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, (n_it - 1) & 1, kBTagDkqDone) &&
+                                             mbar_wait(ctx, bar_drained, 0, kBTagDrained));
     if (ok) {
       tc_fence_after();
-      // Every MMA has completed and every load was consumed: stage dV in the
-      // Q buffers and dK in the dO buffers.
+      // Every MMA has completed, every load was consumed and the dQ drain is
+      // done with the stage buffers: stage dV in the Q buffers and dK in the dO
+      // buffers.
       const uint32_t stV = smem_u32(sQ), stK = smem_u32(sdO);
       const uint32_t tdK = tmem + lane_off + C::kColdK, tdV = tmem + lane_off + C::kColdV;
 #pragma unroll
@@ -448,32 +484,65 @@ __global__ void __launch_bounds__(448, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ dQ drain
+    // Staging: the fp32 dQ tile is 128 rows x D columns = 4 * D * 128 bytes, split
+    // into 32-column boxes (128-byte swizzle); boxes 0..D/64-1 go to Q_i's stage
+    // buffer and the rest to dO_i's (each buffer holds D/64 boxes of 16 KB).
     const int r = (warp & 3) * 32 + lane;  // query row within the tile
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tdQ = tmem + lane_off + C::kColdQ;
+    const bool leader = (warp == 8 && lane == 0);
+    constexpr int kBoxesPerBuf = D / 64;  // 16 KB boxes per stage buffer
     bool ok = !*abort_flag;
     for (int it = 0; it < n_it && ok; ++it) {
+      const int s = it & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, it & 1, kBTagDkqDone));
       if (!ok) break;
       tc_fence_after();
-      const int qrow = (i0 + it) * 128 + r;
-      float *dst = p.ws_dq + (static_cast<size_t>(bh) * p.N + (qrow < p.N ? qrow : 0)) * D;
+      if (r == 0) FA_TRACE(1024 + it * 2 + 0);
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t v[32];
-        tmem_ld32(tdQ + 32 * ch, v);
+      for (int half = 0; half < 2; ++half) {
+        // Columns [half*D/2, (half+1)*D/2) -> the Q (half 0) or dO (half 1) stage buffer.
+        uint32_t v[D / 2];
+#pragma unroll
+        for (int ch = 0; ch < D / 64; ++ch) tmem_ld32(tdQ + half * (D / 2) + 32 * ch, v + 32 * ch);
         tmem_wait_ld();
-        if (qrow < p.N) {
-#pragma unroll
-          for (int t = 0; t < 8; ++t)
-            red_add_v4(dst + 32 * ch + 4 * t, __uint_as_float(v[4 * t]) * p.scale,
-                       __uint_as_float(v[4 * t + 1]) * p.scale, __uint_as_float(v[4 * t + 2]) * p.scale,
-                       __uint_as_float(v[4 * t + 3]) * p.scale);
+        if (half == 1) {
+          tc_fence_before();
+          mbar_arrive(bar_dq_empty);  // dQ is out of TMEM
         }
+        const uint32_t buf = smem_u32((half == 0 ? sQ : sdO) + s * C::kTile);
+#pragma unroll
+        for (int b = 0; b < kBoxesPerBuf; ++b)
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int c0 = 32 * b + 4 * t;
+            st_shared_v4(buf + b * 16384 + bsw128(r, t), __float_as_uint(__uint_as_float(v[c0]) * p.scale),
+                         __float_as_uint(__uint_as_float(v[c0 + 1]) * p.scale),
+                         __float_as_uint(__uint_as_float(v[c0 + 2]) * p.scale),
+                         __float_as_uint(__uint_as_float(v[c0 + 3]) * p.scale));
+          }
       }
-      tc_fence_before();
-      mbar_arrive(bar_dq_empty);
+      fence_proxy_async_smem();
+      mbar_arrive(bar_stage);
+      if (leader) {
+        ok = mbar_wait(ctx, bar_stage, it & 1, kBTagStage);
+        if (ok) {
+          for (int half = 0; half < 2; ++half)
+            for (int b = 0; b < kBoxesPerBuf; ++b)
+              tma_reduce_add_3d(&tmdQacc, (half == 0 ? sQ : sdO) + s * C::kTile + b * 16384,
+                                half * (D / 2) + 32 * b, (i0 + it) * 128, bh);
+          bulk_commit();
+          bulk_wait_read<0>();
+        }
+        // The stage (Q_i, dO_i) is free for the producer: the MMAs that read it
+        // completed (bar_dkq_done) and TMA has read the staged dQ.
+        mbar_arrive(&bar_qdo_empty[s]);
+        if (it == n_it - 1) mbar_arrive(bar_drained);
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      if (r == 0) FA_TRACE(1024 + it * 2 + 1);
     }
+    if (leader) bulk_wait<0>();  // every reduction has landed before the CTA exits
     __syncwarp();
   }
 
@@ -525,10 +594,11 @@ template <int D, bool CAUSAL>
 inline void bwd_main_launch(const CUtensorMap *m, const BwdParams &p, int nkv, cudaStream_t s) {
   const dim3 grid(static_cast<unsigned>(p.BH) * static_cast<unsigned>(nkv));
   fa_bwd_kernel<D, CAUSAL><<<grid, BwdCfg<D>::kThreads, BwdCfg<D>::kSmemBytes, s>>>(m[0], m[1], m[2], m[3], m[4],
-                                                                                      m[5], p);
+                                                                                      m[5], m[6], p);
 }
 
-// maps: Q, K, V, dO, dK, dV (bf16, 3-D, 64-feature boxes).
+// maps: Q, K, V, dO, dK, dV (bf16, 3-D, 64-feature boxes), dQ accumulator
+// (fp32, 3-D, 32-feature boxes).
 inline cudaError_t bwd_launch(const BwdLaunch &L, const CUtensorMap *maps, cudaStream_t s) {
   const int Npad = pad128(L.N);
   float *ws_dq = static_cast<float *>(L.workspace);

@@ -120,9 +120,17 @@ __global__ void __launch_bounds__(352, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work unit: longest-first over query-tile pairs (matters when causal).
-  const int bh = blockIdx.x % p.BH;
-  const int u = p.n_qpairs - 1 - static_cast<int>(blockIdx.x / p.BH);
+  // Work unit: heads in chunks of 8 (their K/V stay resident in L2 while the
+  // chunk runs); inside a chunk, longest query-tile pairs first (causal).
+  int bh, u;
+  {
+    constexpr int kChunk = 8;
+    const int per_chunk = kChunk * p.n_qpairs;
+    const int ch = static_cast<int>(blockIdx.x) / per_chunk, rem = static_cast<int>(blockIdx.x) % per_chunk;
+    const int g = min(kChunk, p.BH - ch * kChunk);
+    u = p.n_qpairs - 1 - rem / g;
+    bh = ch * kChunk + rem % g;
+  }
   const int n_kv_all = (p.N + 127) / 128;
   int n_kv0, n_kv1;  // KV tiles seen by query tile 0 / 1
   if (CAUSAL) {
