@@ -36,8 +36,11 @@ sys.path.insert(0, ROOT)
 METRIC = "attention fwd and fwd+bwd TFLOP/s (bf16, 1×B200) and % of tensor peak"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["io_aware_exact_23_b200/csrc/ptx.cuh", "io_aware_exact_23_b200/csrc/fa_fwd.cuh",
-                  "io_aware_exact_23_b200/csrc/fa_bwd.cuh", "io_aware_exact_23_b200/csrc/fa_api.cu"]
+# Device code of each timed kernel (a changed file invalidates its stored ncu traffic).
+KERNEL_SOURCES = {
+    "fa_fwd_kernel": ["io_aware_exact_23_b200/csrc/ptx.cuh", "io_aware_exact_23_b200/csrc/fa_fwd.cuh"],
+    "fa_bwd_kernel": ["io_aware_exact_23_b200/csrc/ptx.cuh", "io_aware_exact_23_b200/csrc/fa_bwd.cuh"],
+}
 
 
 def parse_args():
@@ -63,9 +66,9 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def source_sha() -> str:
+def source_sha(kernel: str) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES.get(kernel, []):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -79,7 +82,7 @@ def stored_traffic(kernel: str, workload: str):
     with open(p) as f:
         rec = json.load(f)
     for r in rec.get("records", []):
-        if r.get("kernel") == kernel and r.get("workload") == workload and r.get("source_sha") == source_sha():
+        if r.get("kernel") == kernel and r.get("workload") == workload and r.get("source_sha") == source_sha(kernel):
             return r.get("dram_bytes_per_launch")
     return None
 
