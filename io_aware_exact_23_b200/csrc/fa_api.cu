@@ -155,9 +155,10 @@ int device_state(DeviceState **out, int *dev_out) {
 
 template <int D, bool CAUSAL>
 cudaError_t launch_fwd(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v, const CUtensorMap &o,
-                       const fa::FwdParams &p, cudaStream_t stream) {
+                       const CUtensorMap &olo, const fa::FwdParams &p, cudaStream_t stream) {
   const dim3 grid(static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.n_qpairs));
-  fa::fa_fwd_kernel<D, CAUSAL><<<grid, fa::FwdCfg<D>::kThreads, fa::FwdCfg<D>::kSmemBytes, stream>>>(q, k, v, o, p);
+  fa::fa_fwd_kernel<D, CAUSAL><<<grid, fa::FwdCfg<D>::kThreads, fa::FwdCfg<D>::kSmemBytes, stream>>>(q, k, v, o, olo,
+                                                                                                      p);
   return cudaGetLastError();
 }
 
@@ -195,9 +196,9 @@ int fa_fwd_residual(const void *q, const void *k, const void *v, void *o, void *
   if (st != FA_OK) return st;
 
   const int BH = B * H;
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv, to, tolo;
   if (encode_bf16(&tq, q, d, N, BH) || encode_bf16(&tk, k, d, N, BH) || encode_bf16(&tv, v, d, N, BH) ||
-      encode_bf16(&to, o, d, N, BH))
+      encode_bf16(&to, o, d, N, BH) || encode_bf16(&tolo, o_lo ? o_lo : o, d, N, BH))
     return FA_ERR_CUDA;
   fa::FwdParams p;
   p.lse = lse;
@@ -211,9 +212,10 @@ int fa_fwd_residual(const void *q, const void *k, const void *v, void *o, void *
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (d == 64)
-    e = causal ? launch_fwd<64, true>(tq, tk, tv, to, p, s) : launch_fwd<64, false>(tq, tk, tv, to, p, s);
+    e = causal ? launch_fwd<64, true>(tq, tk, tv, to, tolo, p, s) : launch_fwd<64, false>(tq, tk, tv, to, tolo, p, s);
   else
-    e = causal ? launch_fwd<128, true>(tq, tk, tv, to, p, s) : launch_fwd<128, false>(tq, tk, tv, to, p, s);
+    e = causal ? launch_fwd<128, true>(tq, tk, tv, to, tolo, p, s)
+               : launch_fwd<128, false>(tq, tk, tv, to, tolo, p, s);
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

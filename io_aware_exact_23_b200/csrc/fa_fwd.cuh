@@ -59,7 +59,7 @@ struct FwdParams {
 template <int D>
 struct FwdCfg {
   static constexpr int kTileBytes = 128 * D * 2;      // one 128 x D bf16 tile
-  static constexpr int kStages = (D == 128) ? 4 : 8;  // K/V ring depth
+  static constexpr int kStages = (D == 128) ? 4 : 8;  // K/V ring depth (>= 4: the epilogue stages in it)
   static constexpr int kBoxes = D / 64;               // 64-column TMA boxes per tile
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
@@ -98,7 +98,7 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(352, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                  const FwdParams p) {
+                  const __grid_constant__ CUtensorMap tmOlo, const FwdParams p) {
   using C = FwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
 
@@ -396,11 +396,14 @@ __global__ void __launch_bounds__(352, 1)
       }
     }
     // ---------------------------------------------------------- epilogue
+    // Once both tiles' last PV has completed no MMA or load is in flight, so the
+    // K/V ring is free: O_k and its residual are staged there (swizzled) and
+    // written by TMA stores.
+    ok = ok && __all_sync(0xffffffffu, mbar_wait(ctx, &bar_pv_done[0], (n_k[0] - 1) & 1, kTagPvDone) &&
+                                           mbar_wait(ctx, &bar_pv_done[1], (n_k[1] - 1) & 1, kTagPvDone));
+    if (ok) tc_fence_after();
     for (int k = 0; k < 2 && ok; ++k) {
       const int qt = 2 * u + k;
-      ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_pv_done[k], (n_k[k] - 1) & 1, kTagPvDone));
-      if (!ok) break;
-      tc_fence_after();
       // Whole-row sums from the two column halves.
       float *ls = reinterpret_cast<float *>(smem + C::kLOff) + k * 512;  // [h][2][128]
       ls[(h * 2 + 0) * 128 + r] = l[k];
@@ -412,8 +415,8 @@ __global__ void __launch_bounds__(352, 1)
       const float lt = l[k] + ls[((h ^ 1) * 2 + 0) * 128 + r];
       const float lrt = lr[k] + ls[((h ^ 1) * 2 + 1) * 128 + r];
       const float inv_l = 1.f / lrt;
-      uint8_t *stage = sQ + k * C::kTileBytes;  // Q_k is dead: all its MMAs completed
-      const uint32_t stage_addr = smem_u32(stage);
+      const uint32_t st_o = smem_u32(sKV + (2 * k) * C::kTileBytes);
+      const uint32_t st_lo = smem_u32(sKV + (2 * k + 1) * C::kTileBytes);
       const uint32_t tO = tmem + lane_off + 256 + k * D;
 #pragma unroll
       for (int ch = 0; ch < D / 64; ++ch) {
@@ -425,36 +428,46 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
         for (int t = 0; t < 16; ++t)
           w[t] = pack_bf16(__uint_as_float(o[2 * t]) * inv_l, __uint_as_float(o[2 * t + 1]) * inv_l);
-        if (p.o_lo != nullptr && qt * 128 + r < p.N) {
-          // What rounding O to bf16 dropped, itself rounded to bf16: O ~ o + o_lo
-          // to about 16 significant bits (used by the backward's D = rowsum(dO o O)).
-          uint32_t lo[16];
-#pragma unroll
-          for (int t = 0; t < 16; ++t) {
-            const float a = __uint_as_float(o[2 * t]) * inv_l, b = __uint_as_float(o[2 * t + 1]) * inv_l;
-            lo[t] = pack_bf16(a - __uint_as_float(w[t] << 16), b - __uint_as_float(w[t] & 0xFFFF0000u));
-          }
-          uint4 *dst = reinterpret_cast<uint4 *>(p.o_lo + (static_cast<size_t>(bh) * p.N + qt * 128 + r) * D + col0);
-#pragma unroll
-          for (int t = 0; t < 4; ++t) dst[t] = make_uint4(lo[4 * t], lo[4 * t + 1], lo[4 * t + 2], lo[4 * t + 3]);
-        }
         const int box = col0 >> 6, chunk0 = (col0 & 63) >> 3;
 #pragma unroll
         for (int t = 0; t < 4; ++t)
-          st_shared_v4(stage_addr + box * 16384 + sw128_offset(r, chunk0 + t), w[4 * t], w[4 * t + 1],
-                       w[4 * t + 2], w[4 * t + 3]);
+          st_shared_v4(st_o + box * 16384 + sw128_offset(r, chunk0 + t), w[4 * t], w[4 * t + 1], w[4 * t + 2],
+                       w[4 * t + 3]);
+        if (p.o_lo != nullptr) {
+          // What rounding O to bf16 dropped, itself rounded to bf16: O ~ o + o_lo
+          // to about 16 significant bits (used by the backward's D = rowsum(dO o O)).
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const float a = __uint_as_float(o[2 * t]) * inv_l, b = __uint_as_float(o[2 * t + 1]) * inv_l;
+            w[t] = pack_bf16(a - __uint_as_float(w[t] << 16), b - __uint_as_float(w[t] & 0xFFFF0000u));
+          }
+#pragma unroll
+          for (int t = 0; t < 4; ++t)
+            st_shared_v4(st_lo + box * 16384 + sw128_offset(r, chunk0 + t), w[4 * t], w[4 * t + 1], w[4 * t + 2],
+                         w[4 * t + 3]);
+        }
       }
       const int grow = qt * 128 + r;
       if (h == 0 && grow < p.N) p.lse[static_cast<size_t>(bh) * p.N + grow] = (m[k] + log2f(lt)) * 0.69314718055994531f;
-      // Make the generic-proxy smem writes visible to TMA, then one thread
-      // stores the tile once all softmax threads have written their part.
+    }
+    // Make the generic-proxy smem writes visible to TMA, then one thread stores
+    // both tiles once all softmax threads have written their part.
+    if (ok) {
       fence_proxy_async_smem();
-      mbar_arrive(&bar_epi[k]);
-      if (warp == 0 && lane == 0 && mbar_wait(ctx, &bar_epi[k], 0, kTagEpi) && qt * 128 < p.N) {
-        for (int b = 0; b < C::kBoxes; ++b) tma_store_3d(&tmO, stage + b * 16384, b * 64, qt * 128, bh);
+      mbar_arrive(&bar_epi[0]);
+      if (warp == 0 && lane == 0 && mbar_wait(ctx, &bar_epi[0], 0, kTagEpi)) {
+        for (int k = 0; k < 2; ++k) {
+          const int qt = 2 * u + k;
+          if (qt * 128 >= p.N) continue;
+          for (int b = 0; b < C::kBoxes; ++b) {
+            tma_store_3d(&tmO, sKV + (2 * k) * C::kTileBytes + b * 16384, b * 64, qt * 128, bh);
+            if (p.o_lo != nullptr)
+              tma_store_3d(&tmOlo, sKV + (2 * k + 1) * C::kTileBytes + b * 16384, b * 64, qt * 128, bh);
+          }
+        }
         bulk_commit();
         bulk_wait_read<0>();
-        FA_TRACE(6 + k);
+        FA_TRACE(6);
       }
     }
     __syncwarp();
