@@ -22,8 +22,9 @@
 // TMEM columns (512 allocated): S0 [0,128), S1 [128,256), O0 [256,256+D),
 // O1 [256+D, 256+2D).  The bf16 P (two per column) of column half h is written
 // over S columns [64h, 64h+32) -- inside the half its warp has already read --
-// and is the A operand of the PV MMA straight from TMEM.  So the next S of a
-// tile is issued only once that tile's PV has completed.
+// and is the A operand of the PV MMA straight from TMEM.  The next S of a tile
+// overwrites those columns; its issuer puts it in the pipe right behind that
+// tile's PV (one issuing thread: the MMAs execute in order), without waiting.
 //
 // Online softmax, in the log2 domain with c = scale*log2(e):
 //   m' = max(m, c*rowmax(S));  P = 2^(c*S - m');  l = 2^(m-m') l + rowsum(P);
@@ -246,10 +247,9 @@ __global__ void __launch_bounds__(352, 1)
           if (ok) mbar_arrive(&bar_kv_empty[sV]);
           continue;
         }
-        // S_k aliases P_k: the previous PV_k must have consumed P_k.
-        if (j > 0) ok = mbar_wait(ctx, &bar_pv_done[k], (j - 1) & 1, kTagPvDone);
-        if (!ok) break;
-        tc_fence_after();
+        // S_k aliases P_k, which the previous PV_k reads.  Both MMAs come from
+        // this thread and the tensor pipe runs them in issue order, so S_k is
+        // issued right behind PV_k without waiting for it to complete.
         const uint64_t k_desc = sdesc_add(k_desc0, sK * C::kTileBytes);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
