@@ -37,9 +37,10 @@
 // After the first KV step P is computed against the running max before the
 // row max of the new tile is known (the half maxima travel through smem in the
 // meantime); only a row whose max grew by more than 8 recomputes its P.
-// One pair in four of the exponentials runs on the FMA pipe (a cubic after
-// range reduction) instead of the MUFU unit, which is otherwise the bottleneck
-// (one exp per 4d FLOPs; at d = 128 the MUFU rate equals the tensor rate).
+// Every exponential runs on the MUFU unit (one per 4d FLOPs; at d = 128 its
+// rate equals the tensor rate).  Moving a share of them to the FMA pipe as a
+// polynomial was measured slower: FP32-pipe pressure from the softmax warps
+// delays the MMA issue more than the MUFU queue does.
 #pragma once
 
 #include "ptx.cuh"
@@ -67,9 +68,10 @@ struct FwdCfg {
   static constexpr int kXOff = kKVOff + kStages * kTileBytes;  // half-row maxima [2 tiles][2 halves][128]
   static constexpr int kLOff = kXOff + 2048;                   // half-row sums [2 tiles][2 halves][2][128]
   static constexpr int kBarOff = kLOff + 4096;
-  // mbarriers: q[2], kv_full/kv_empty[kStages], then 8 pairs; then the TMEM
-  // address slot and the abort flag.
-  static constexpr int kNumBars = 2 + 2 * kStages + 16;
+  // mbarriers: q[2], kv_full/kv_empty[kStages], s_full/p_full/pv_done/epi/
+  // drain [2] each (one per query tile), the max and sum exchanges [2][4] (one
+  // per tile and warp pair), two spare; then the TMEM address slot and the abort flag.
+  static constexpr int kNumBars = 2 + 2 * kStages + 26;
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kThreads = 352;
   static constexpr int kSoftmaxThreads = 256;
@@ -112,10 +114,10 @@ __global__ void __launch_bounds__(352, 1)
   uint64_t *bar_pv_done = bar_p_full + 2;            // [2] PV_k completed
   uint64_t *bar_epi = bar_pv_done + 2;               // [2]
   uint64_t *bar_drain = bar_epi + 2;                 // [2]
-  uint64_t *bar_x = bar_drain + 2;                   // [2] half-row max exchange
-  uint64_t *bar_l = bar_x + 2;                       // [2] half-row sum exchange
-  static_assert(2 + 2 * C::kStages + 16 == C::kNumBars, "barrier count");
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_l + 2);
+  uint64_t *bar_x = bar_drain + 2;                   // [2][4] half-row max exchange, per warp pair
+  uint64_t *bar_l = bar_x + 8;                       // [2][4] half-row sum exchange, per warp pair
+  static_assert(2 + 2 * C::kStages + 26 == C::kNumBars, "barrier count");
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_l + 8);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -161,8 +163,11 @@ __global__ void __launch_bounds__(352, 1)
       mbar_init(&bar_p_full[k], C::kSoftmaxThreads);
       mbar_init(&bar_pv_done[k], 1);
       mbar_init(&bar_epi[k], C::kSoftmaxThreads);
-      mbar_init(&bar_x[k], C::kSoftmaxThreads);
-      mbar_init(&bar_l[k], C::kSoftmaxThreads);
+      for (int q = 0; q < 4; ++q) {
+        // Warps q and q+4 share rows 32q..32q+31 (and an SM sub-partition).
+        mbar_init(&bar_x[k * 4 + q], 64);
+        mbar_init(&bar_l[k * 4 + q], 64);
+      }
       mbar_init(&bar_drain[k], 1);
     }
     fence_barrier_init();
@@ -314,15 +319,16 @@ __global__ void __launch_bounds__(352, 1)
           for (int cc = 0; cc < 64; ++cc)
             if (cc >= nv) s[cc] = __float_as_uint(-INFINITY);
         }
-        float ma = __uint_as_float(s[0]), mb = __uint_as_float(s[32]);
+        // Half-row max as a shallow tree (eight independent chains of four).
+        float mq[8];
 #pragma unroll
-        for (int t = 1; t < 31; t += 2) {
-          ma = fmax3(ma, __uint_as_float(s[t]), __uint_as_float(s[t + 1]));
-          mb = fmax3(mb, __uint_as_float(s[32 + t]), __uint_as_float(s[33 + t]));
+        for (int q = 0; q < 8; ++q) {
+          const float *v = reinterpret_cast<const float *>(s + 8 * q);
+          mq[q] = fmaxf(fmax3(fmax3(fmax3(v[0], v[1], v[2]), v[3], v[4]), v[5], v[6]), v[7]);
         }
-        const float mh = fmax3(ma, mb, fmaxf(__uint_as_float(s[31]), __uint_as_float(s[63])));
+        const float mh = fmax3(fmax3(mq[0], mq[1], mq[2]), fmax3(mq[3], mq[4], mq[5]), fmaxf(mq[6], mq[7]));
         xm[(k * 2 + h) * 128 + r] = mh;
-        mbar_arrive(&bar_x[k]);
+        mbar_arrive(&bar_x[k * 4 + rq]);
         // P = 2^(c*S - m) for this half row, with the row sums of P in fp32
         // (for the LSE) and of P rounded to bf16 (the PV weights; O's normaliser).
         uint32_t pk[32];
@@ -334,14 +340,9 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
           for (int cc = 0; cc < 32; ++cc) {
             const uint64_t x2 = ffma2(f2pack(__uint_as_float(s[2 * cc]), __uint_as_float(s[2 * cc + 1])), c2, n2);
-            float x0, x1, a, b;
+            float x0, x1;
             f2unpack(x2, x0, x1);
-            if ((cc & 3) == 3) {
-              exp2_poly_pair(x0, x1, a, b);
-            } else {
-              a = ex2(x0);
-              b = ex2(x1);
-            }
+            const float a = ex2(x0), b = ex2(x1);
             acc[cc & 1] = fadd2(acc[cc & 1], f2pack(a, b));
             pk[cc] = pack_bf16(a, b);
             racc[cc & 1] =
@@ -357,7 +358,7 @@ __global__ void __launch_bounds__(352, 1)
         };
         const float m_old = m[k];
         if (m_old != -INFINITY) exps(m_old);  // optimistic: the running max usually holds
-        ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_x[k], j & 1, kTagXmax));
+        ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_x[k * 4 + rq], j & 1, kTagXmax));
         if (!ok) break;
         const float m_cand = fmaxf(mh, xm[(k * 2 + (h ^ 1)) * 128 + r]) * c;
         float alpha = 1.f;
@@ -408,8 +409,8 @@ __global__ void __launch_bounds__(352, 1)
       float *ls = reinterpret_cast<float *>(smem + C::kLOff) + k * 512;  // [h][2][128]
       ls[(h * 2 + 0) * 128 + r] = l[k];
       ls[(h * 2 + 1) * 128 + r] = lr[k];
-      mbar_arrive(&bar_l[k]);
-      ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_l[k], 0, kTagLsum));
+      mbar_arrive(&bar_l[k * 4 + rq]);
+      ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_l[k * 4 + rq], 0, kTagLsum));
       if (!ok) break;
       if (r == 0 && h == 0) FA_TRACE(4 + k);
       const float lt = l[k] + ls[((h ^ 1) * 2 + 0) * 128 + r];

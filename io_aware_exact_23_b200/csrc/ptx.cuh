@@ -330,35 +330,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// Software 2^x for a pair, on the FMA pipe (relieves the MUFU unit):
-// 2^x = 2^n * p(f) with n = rint(x), f = x - n in [-1/2, 1/2] and p the cubic
-// minimax fit of 2^f on that interval (relative error 7.5e-5; coefficients from
-// csrc/gen_exp2_poly.py, a Remez fit of our own).  n is read from the low bits
-// of x + 1.5*2^23 and added to p's exponent field.  Inputs are clamped at -126
-// (so n >= -126 and the exponent field stays >= 0: masked -inf entries give a
-// positive value below 2^-125 instead of 0).  Inputs above 127 are not expected.
-__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float &y0, float &y1) {
-  const uint64_t kMagic = f2pack(12582912.f, 12582912.f);
-  const uint64_t kNegMagic = f2pack(-12582912.f, -12582912.f);
-  const uint64_t kNegOne = f2pack(-1.f, -1.f);
-  const uint64_t c0 = f2pack(0.9999280571937561f, 0.9999280571937561f);
-  const uint64_t c1 = f2pack(0.6932609677314758f, 0.6932609677314758f);
-  const uint64_t c2 = f2pack(0.2426111251115799f, 0.2426111251115799f);
-  const uint64_t c3 = f2pack(0.0551716685295105f, 0.0551716685295105f);
-  const uint64_t x = f2pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
-  const uint64_t t = fadd2(x, kMagic);          // rint(x) in the low mantissa bits
-  const uint64_t r = fadd2(t, kNegMagic);       // rint(x) as a float
-  const uint64_t f = ffma2(r, kNegOne, x);      // x - rint(x), exact
-  uint64_t pp = ffma2(f, c3, c2);
-  pp = ffma2(pp, f, c1);
-  pp = ffma2(pp, f, c0);
-  float p0, p1, t0, t1;
-  f2unpack(pp, p0, p1);
-  f2unpack(t, t0, t1);
-  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
-
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` lands in bits 0..15.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
