@@ -106,51 +106,62 @@ __device__ __forceinline__ uint32_t bsw128(int row, int chunk) {
 // ----------------------------------------------------------- preprocess
 // Lanes-per-row = D / 8 (each lane handles 8 features = 16 bytes).
 template <int D>
-__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t *__restrict__ o,
+__global__ void __launch_bounds__(256, 4) fa_bwd_pre_kernel(const uint16_t *__restrict__ o,
                                                          const uint16_t *__restrict__ o_lo,
                                                          const uint16_t *__restrict__ dO,
                                                          const float *__restrict__ lse, float *__restrict__ ws_D,
                                                          float *__restrict__ ws_lse2, float *__restrict__ ws_dq,
                                                          int N, int Npad, int BH) {
-  constexpr int LPR = D / 8;
+  constexpr int LPR = D / 8;     // lanes per row, 16 bytes each
   constexpr int RPW = 32 / LPR;  // rows per warp pass
+  constexpr int U = 4;           // passes whose loads are in flight together
   const int lane = threadIdx.x & 31;
   const int sub = lane / LPR, part = lane % LPR;
   const long warps = static_cast<long>(gridDim.x) * (blockDim.x / 32);
   const long gw = static_cast<long>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
   const long rows = static_cast<long>(BH) * Npad;
-  for (long base = gw * RPW; base < rows; base += warps * RPW) {
-    const long row = base + sub;
-    float acc = 0.f;
-    const bool in = row < rows;
-    const int bh = in ? static_cast<int>(row / Npad) : 0;
-    const int i = in ? static_cast<int>(row % Npad) : 0;
-    const bool valid = in && i < N;
-    if (valid) {
-      const size_t off = (static_cast<size_t>(bh) * N + i) * D + part * 8;
-      const uint4 a = *reinterpret_cast<const uint4 *>(o + off);
-      const uint4 b = *reinterpret_cast<const uint4 *>(dO + off);
-      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+  const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+  for (long base = gw * RPW * U; base < rows; base += warps * RPW * U) {
+    uint4 a[U], b[U], c[U];
+    bool valid[U];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        acc = fmaf(__uint_as_float(av[t] << 16), __uint_as_float(bv[t] << 16), acc);
-        acc = fmaf(__uint_as_float(av[t] & 0xFFFF0000u), __uint_as_float(bv[t] & 0xFFFF0000u), acc);
-      }
-      if (o_lo != nullptr) {
-        const uint4 c = *reinterpret_cast<const uint4 *>(o_lo + off);
-        const uint32_t cv[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          acc = fmaf(__uint_as_float(cv[t] << 16), __uint_as_float(bv[t] << 16), acc);
-          acc = fmaf(__uint_as_float(cv[t] & 0xFFFF0000u), __uint_as_float(bv[t] & 0xFFFF0000u), acc);
-        }
+    for (int u = 0; u < U; ++u) {
+      const long row = base + u * RPW + sub;
+      const int bh = row < rows ? static_cast<int>(row / Npad) : 0;
+      const int i = row < rows ? static_cast<int>(row % Npad) : 0;
+      valid[u] = row < rows && i < N;
+      a[u] = b[u] = c[u] = zero4;
+      if (valid[u]) {
+        const size_t off = (static_cast<size_t>(bh) * N + i) * D + part * 8;
+        a[u] = *reinterpret_cast<const uint4 *>(o + off);
+        b[u] = *reinterpret_cast<const uint4 *>(dO + off);
+        if (o_lo != nullptr) c[u] = *reinterpret_cast<const uint4 *>(o_lo + off);
       }
     }
 #pragma unroll
-    for (int w = LPR / 2; w >= 1; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
-    if (in && part == 0) {
-      ws_D[row] = valid ? acc : 0.f;
-      ws_lse2[row] = valid ? lse[static_cast<size_t>(bh) * N + i] * 1.4426950408889634f : INFINITY;
+    for (int u = 0; u < U; ++u) {
+      const uint32_t av[4] = {a[u].x, a[u].y, a[u].z, a[u].w}, bv[4] = {b[u].x, b[u].y, b[u].z, b[u].w};
+      const uint32_t cv[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+      float acc = 0.f;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        // O = o + o_lo when the forward wrote its rounding residual.
+        const float b_lo = __uint_as_float(bv[t] << 16), b_hi = __uint_as_float(bv[t] & 0xFFFF0000u);
+        acc = fmaf(__uint_as_float(av[t] << 16), b_lo, acc);
+        acc = fmaf(__uint_as_float(av[t] & 0xFFFF0000u), b_hi, acc);
+        if (o_lo != nullptr) {
+          acc = fmaf(__uint_as_float(cv[t] << 16), b_lo, acc);
+          acc = fmaf(__uint_as_float(cv[t] & 0xFFFF0000u), b_hi, acc);
+        }
+      }
+#pragma unroll
+      for (int w = LPR / 2; w >= 1; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
+      const long row = base + u * RPW + sub;
+      if (row < rows && part == 0) {
+        const int bh = static_cast<int>(row / Npad), i = static_cast<int>(row % Npad);
+        ws_D[row] = valid[u] ? acc : 0.f;
+        ws_lse2[row] = valid[u] ? lse[static_cast<size_t>(bh) * N + i] * 1.4426950408889634f : INFINITY;
+      }
     }
   }
   const long n4 = static_cast<long>(BH) * N * D / 4;
@@ -163,13 +174,23 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t *__restr
 // --------------------------------------------------------- dQ conversion
 __global__ void __launch_bounds__(256) fa_dq_convert_kernel(const float *__restrict__ ws_dq,
                                                             uint16_t *__restrict__ dq, long n4) {
+  constexpr int U = 4;  // loads in flight per thread
   const long tid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long nthreads = static_cast<long>(gridDim.x) * blockDim.x;
   const float4 *src = reinterpret_cast<const float4 *>(ws_dq);
   uint2 *dst = reinterpret_cast<uint2 *>(dq);
-  for (long t = tid; t < n4; t += nthreads) {
-    const float4 v = src[t];
-    dst[t] = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+  for (long t0 = tid; t0 < n4; t0 += nthreads * U) {
+    float4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long t = t0 + u * nthreads;
+      v[u] = t < n4 ? __ldcs(src + t) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long t = t0 + u * nthreads;
+      if (t < n4) dst[t] = make_uint2(pack_bf16(v[u].x, v[u].y), pack_bf16(v[u].z, v[u].w));
+    }
   }
 }
 
@@ -604,7 +625,7 @@ inline cudaError_t bwd_launch(const BwdLaunch &L, const CUtensorMap *maps, cudaS
   float *ws_dq = static_cast<float *>(L.workspace);
   float *ws_lse2 = ws_dq + static_cast<size_t>(L.BH) * L.N * L.d;
   float *ws_D = ws_lse2 + static_cast<size_t>(L.BH) * Npad;
-  const int pre_grid = L.num_sms * 4;
+  const int pre_grid = L.num_sms * 8;
   cudaError_t e = cudaSuccess;
   if (L.events && (e = cudaEventRecord(L.events[0], s)) != cudaSuccess) return e;
   if (L.d == 64)
