@@ -46,7 +46,7 @@ KERNEL_SOURCES = {
 def parse_args():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="b2h32n4096d128_causal")
@@ -112,6 +112,12 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.samples.append((time.time(), line.strip()))
 
+    def wait_ready(self, timeout: float = 10.0):
+        """Block until nvidia-smi has produced its first sample (or timeout)."""
+        t_end = time.time() + timeout
+        while self.proc is not None and not self.samples and time.time() < t_end:
+            time.sleep(0.02)
+
     def stop(self):
         if self.proc is not None:
             self.proc.terminate()
@@ -121,6 +127,11 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self, t0: float, t1: float):
+        # Samples inside the timed region; if it was shorter than the sampling
+        # period, the samples within a quarter second of it.
+        window = "timed region"
+        if not any(t0 <= ts <= t1 for ts, _ in self.samples):
+            t0, t1, window = t0 - 0.25, t1 + 0.25, "timed region +-0.25 s"
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ts, line in self.samples:
@@ -140,7 +151,7 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "window": window}
 
 
 def dist_setup():
@@ -293,7 +304,7 @@ def main():
     except Exception:
         pass
     sampler = ClockSampler(uuid)
-    time.sleep(0.3)
+    sampler.wait_ready()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()

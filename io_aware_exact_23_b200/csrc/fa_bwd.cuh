@@ -34,7 +34,8 @@
 //                 dK  += dS^T Q_i       (smem x smem)
 //                 dQ_i = dS K_j         (smem x smem, dS read transposed)
 //
-// TMEM columns (512): S^T [0,128) with P^T (bf16) over its first 64 columns;
+// TMEM columns (512): S^T [0,128) with P^T (bf16) of query columns 64w..64w+63
+// over S^T columns [64w, 64w+32) (w = 0, 1: the half each compute warp reads);
 // dP^T [128,256); dK [256,256+D); dV [256+D,256+2D); dQ reuses dP^T's columns
 // when D = 128 (dP^T is dead once dS is formed) and [384,448) when D = 64.
 // dS^T (bf16) is written to smem in the 128-byte-swizzled K-major layout,
@@ -212,7 +213,7 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t *bar_dp_full = bars + 6;
   uint64_t *bar_p_full = bars + 7;
   uint64_t *bar_ds_full = bars + 8;
-  uint64_t *bar_dv_done = bars + 9;
+  uint64_t *bar_spare = bars + 9;     // unused
   uint64_t *bar_dkq_done = bars + 10;
   uint64_t *bar_dq_empty = bars + 11;
   uint64_t *bar_epi = bars + 12;
@@ -253,7 +254,7 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(bar_dp_full, 1);
     mbar_init(bar_p_full, 256);
     mbar_init(bar_ds_full, 256);
-    mbar_init(bar_dv_done, 1);
+    mbar_init(bar_spare, 1);
     mbar_init(bar_dkq_done, 1);
     mbar_init(bar_dq_empty, 128);
     mbar_init(bar_epi, 256);
@@ -327,15 +328,8 @@ __global__ void __launch_bounds__(448, 1)
       const uint64_t dOk0 = make_sdesc(smem_u32(sdO), 16, 1024), dOm0 = make_sdesc(smem_u32(sdO), 16384, 1024);
       const uint32_t tS = tmem + C::kColS, tdP = tmem + C::kColdP, tdK = tmem + C::kColdK;
       const uint32_t tdV = tmem + C::kColdV, tdQ = tmem + C::kColdQ;
-      bool ok = mbar_wait(ctx, bar_kv, 0, kBTagKV);
-      for (int it = 0; it < n_it && ok; ++it) {
-        const int s = it & 1, n = it >> 1;
-        const uint64_t dQk = sdesc_add(dQk0, s * C::kTile), dQm = sdesc_add(dQm0, s * C::kTile);
-        const uint64_t dOk = sdesc_add(dOk0, s * C::kTile), dOm = sdesc_add(dOm0, s * C::kTile);
-        ok = mbar_wait(ctx, &bar_qdo_full[s], n & 1, kBTagQdoFull);
-        if (ok && it > 0) ok = mbar_wait(ctx, bar_dv_done, (it - 1) & 1, kBTagDvDone);
-        if (!ok) break;
-        tc_fence_after();
+      auto issue_sT = [&](int it) {  // S^T = K_j Q_i^T
+        const uint64_t dQk = sdesc_add(dQk0, (it & 1) * C::kTile);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
@@ -343,11 +337,9 @@ __global__ void __launch_bounds__(448, 1)
         }
         mma_commit(bar_s_full);
         FA_TRACE(16 + it * 8 + 0);
-        if (D == 128 && it > 0) {
-          ok = mbar_wait(ctx, bar_dq_empty, (it - 1) & 1, kBTagDqEmpty);
-          if (!ok) break;
-          tc_fence_after();
-        }
+      };
+      auto issue_dPT = [&](int it) {  // dP^T = V_j dO_i^T
+        const uint64_t dOk = sdesc_add(dOk0, (it & 1) * C::kTile);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
@@ -355,32 +347,94 @@ __global__ void __launch_bounds__(448, 1)
         }
         mma_commit(bar_dp_full);
         FA_TRACE(16 + it * 8 + 1);
-        ok = mbar_wait(ctx, bar_p_full, it & 1, kBTagPFull);
-        if (!ok) break;
-        tc_fence_after();
+      };
+      auto issue_dV = [&](int it) {  // dV += P^T dO_i; P^T of query columns 64w.. at S^T columns 64w..64w+31
+        const uint64_t dOm = sdesc_add(dOm0, (it & 1) * C::kTile);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_ts(tdV, tS + ks * 8, sdesc_add(dOm, ks * 2048), id_kxmn, (it > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(bar_dv_done);
+          mma_ts(tdV, tS + ks * 8 + (ks >= 4 ? 32 : 0), sdesc_add(dOm, ks * 2048), id_kxmn,
+                 (it > 0 || ks > 0) ? 1u : 0u);
         FA_TRACE(16 + it * 8 + 2);
-        ok = mbar_wait(ctx, bar_ds_full, it & 1, kBTagDsFull);
-        if (!ok) break;
-        tc_fence_after();
+      };
+      auto issue_dK = [&](int it) {  // dK += dS^T Q_i
+        const uint64_t dQm = sdesc_add(dQm0, (it & 1) * C::kTile);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
           mma_ss(tdK, sdesc_add(dSk, off), sdesc_add(dQm, ks * 2048), id_kxmn, (it > 0 || ks > 0) ? 1u : 0u);
         }
-        if (D == 64 && it > 0) {
-          ok = mbar_wait(ctx, bar_dq_empty, (it - 1) & 1, kBTagDqEmpty);
-          if (!ok) break;
-          tc_fence_after();
-        }
+      };
+      auto issue_dQ = [&](int it) {  // dQ_i = dS K_j; the dQ drain releases the Q/dO stage after staging through it
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           mma_ss(tdQ, sdesc_add(dSm, ks * 2048), sdesc_add(dKm, ks * 2048), id_mnmn, ks > 0);
-        mma_commit(bar_dkq_done);  // the dQ drain releases the Q/dO stage after staging through it
+        mma_commit(bar_dkq_done);
         FA_TRACE(16 + it * 8 + 3);
+      };
+      auto wait_stage = [&](int it) {
+        return mbar_wait(ctx, &bar_qdo_full[it & 1], (it >> 1) & 1, kBTagQdoFull);
+      };
+      // S^T(i+1) overwrites P^T(i), which dV(i) reads, and dP^T(i+1) the dP^T(i)
+      // the compute warps have turned into dS(i): neither waits for an MMA to
+      // complete, since one thread issues them all and the pipe runs them in order.
+      bool ok = mbar_wait(ctx, bar_kv, 0, kBTagKV);
+      if (D == 128) {
+        // Order S^T(i) dP^T(i) dV(i) dK(i) dQ(i).  dQ(i) accumulates in dP^T's
+        // columns, so dP^T(i+1) also waits for the drain to have read dQ(i).
+        for (int it = 0; it < n_it && ok; ++it) {
+          ok = wait_stage(it);
+          if (!ok) break;
+          tc_fence_after();
+          issue_sT(it);
+          if (it > 0) {
+            ok = mbar_wait(ctx, bar_dq_empty, (it - 1) & 1, kBTagDqEmpty);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          issue_dPT(it);
+          ok = mbar_wait(ctx, bar_p_full, it & 1, kBTagPFull);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dV(it);
+          ok = mbar_wait(ctx, bar_ds_full, it & 1, kBTagDsFull);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dK(it);
+          issue_dQ(it);
+        }
+      } else {
+        // Order S^T(0) dP^T(0) | dV(i) S^T(i+1) dK(i) dQ(i) dP^T(i+1) | ...: the
+        // next tile's S^T goes in ahead of dK(i) / dQ(i) (dQ has columns of its
+        // own), so the compute warps start tile i+1 while those run.
+        ok = ok && wait_stage(0);
+        if (ok) {
+          tc_fence_after();
+          issue_sT(0);
+          issue_dPT(0);
+        }
+        for (int it = 0; it < n_it && ok; ++it) {
+          ok = mbar_wait(ctx, bar_p_full, it & 1, kBTagPFull);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dV(it);
+          if (it + 1 < n_it) {
+            ok = wait_stage(it + 1);
+            if (!ok) break;
+            tc_fence_after();
+            issue_sT(it + 1);
+          }
+          ok = mbar_wait(ctx, bar_ds_full, it & 1, kBTagDsFull);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dK(it);
+          if (it > 0) {  // dQ(i-1) has left its columns
+            ok = mbar_wait(ctx, bar_dq_empty, (it - 1) & 1, kBTagDqEmpty);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          issue_dQ(it);
+          if (it + 1 < n_it) issue_dPT(it + 1);
+        }
       }
       if (!ok) {
         mma_commit(bar_drain);
@@ -423,7 +477,7 @@ __global__ void __launch_bounds__(448, 1)
       uint32_t pk[32];
 #pragma unroll
       for (int t = 0; t < 32; ++t) pk[t] = pack_bf16(pf[2 * t], pf[2 * t + 1]);
-      tmem_st32(tS + 32 * w, pk);
+      tmem_st32(tS + 64 * w, pk);  // inside the columns this warp has read
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p_full);
