@@ -18,6 +18,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfa.so")
+# Standard-attention baseline (cuBLAS GEMMs + its own row kernels), kept out of libfa.so.
+VANILLA_LIB = os.path.join(PKG, "libfa_vanilla.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -44,6 +46,26 @@ def needs_build() -> bool:
     return any(os.path.getmtime(p) > t for p in deps())
 
 
+def vanilla_deps():
+    return [os.path.join(CSRC, "vanilla.cu"), os.path.join(INCLUDE, "fa.h"), os.path.join(INCLUDE, "fa_vanilla.h")]
+
+
+def build_vanilla(force: bool = False, verbose: bool = False) -> str:
+    """Compile libfa_vanilla.so (links cuBLAS)."""
+    if not force and os.path.exists(VANILLA_LIB) and all(
+            os.path.getmtime(p) <= os.path.getmtime(VANILLA_LIB) for p in vanilla_deps()):
+        return VANILLA_LIB
+    tmp = VANILLA_LIB + f".tmp{os.getpid()}"
+    cmd = [nvcc_path(), *ARCH, "-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
+           "-I", INCLUDE, os.path.join(CSRC, "vanilla.cu"), "-lcublas", "-o", tmp]
+    if verbose:
+        cmd.insert(1, "-Xptxas=-v")
+        print(" ".join(cmd), flush=True)
+    subprocess.check_call(cmd)
+    os.replace(tmp, VANILLA_LIB)
+    return VANILLA_LIB
+
+
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if not force and not needs_build():
         return LIB
@@ -64,4 +86,5 @@ if __name__ == "__main__":
     ap.add_argument("-v", "--verbose", action="store_true", help="print the command and ptxas resource usage")
     a = ap.parse_args()
     print(build(force=a.force, verbose=a.verbose))
+    print(build_vanilla(force=a.force, verbose=a.verbose))
     sys.exit(0)
