@@ -24,17 +24,18 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "ref_attn.c")
+_SRCS = [_SRC, os.path.join(_HERE, "ref_dropout.c")]
 _LIB = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile ``ref_attn.c`` into ``liboracle.so`` (plain -O2, IEEE fp64)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    """Compile ``ref_attn.c`` and ``ref_dropout.c`` into ``liboracle.so`` (plain -O2, IEEE fp64)."""
+    if force or not os.path.exists(_LIB) or any(os.path.getmtime(_LIB) < os.path.getmtime(s) for s in _SRCS):
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.check_call(
             ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
-             "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"])
+             "-fno-fast-math", "-ffp-contract=off", *_SRCS, "-o", tmp, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -54,6 +55,16 @@ def _load():
         for f in (lib.ref_attn_fwd, lib.ref_attn_bwd, lib.ref_attn_fwd_rows, lib.ref_attn_dq_rows,
                   lib.ref_attn_dkdv_rows):
             f.restype = ctypes.c_int
+        U32 = ctypes.POINTER(ctypes.c_uint32)
+        u64, u32 = ctypes.c_uint64, ctypes.c_uint32
+        lib.ref_philox4x32_10.argtypes = [U32, U32, U32]
+        lib.ref_philox4x32_10.restype = None
+        lib.ref_dropout_mask.argtypes = [cl, cl, u64, u32, u32, ctypes.POINTER(ctypes.c_uint8)]
+        lib.ref_dropout_mask.restype = None
+        lib.ref_attn_fwd_dropout.argtypes = [D, D, D, D, D, cl, cl, cl, cd, ci, u64, u32, u32]
+        lib.ref_attn_fwd_dropout.restype = ci
+        lib.ref_attn_bwd_dropout.argtypes = [D, D, D, D, D, D, D, cl, cl, cl, cd, ci, u64, u32, u32]
+        lib.ref_attn_bwd_dropout.restype = ci
         _lib = lib
     return _lib
 
@@ -158,3 +169,54 @@ def ref_dkdv_rows(q, k, v, dO, scale: float, causal: bool, head: int, key_rows, 
     if rc != 0:
         raise RuntimeError(f"ref_attn_dkdv_rows failed ({rc})")
     return dk, dv
+
+
+# ------------------------------------------------------------------ dropout
+
+def dropout_threshold(rate: float) -> int:
+    """T = floor(rate * 65536): a key is dropped when its 16-bit draw is below T."""
+    if not (0.0 <= rate < 1.0):
+        raise ValueError("dropout rate must be in [0, 1)")
+    return int(np.floor(float(rate) * 65536.0))
+
+
+def philox4x32_10(counter, key):
+    """Philox4x32-10 of a 4-word counter and a 2-word key (``ref_dropout.c``)."""
+    c = (ctypes.c_uint32 * 4)(*[int(x) & 0xFFFFFFFF for x in counter])
+    k = (ctypes.c_uint32 * 2)(*[int(x) & 0xFFFFFFFF for x in key])
+    out = (ctypes.c_uint32 * 4)()
+    _load().ref_philox4x32_10(c, k, out)
+    return [int(x) for x in out]
+
+
+def dropout_mask(BH: int, N: int, seed: int, offset: int, rate: float) -> np.ndarray:
+    """keep[bh, i, j] (uint8 0/1) of the dropout mask, [BH, N, N]."""
+    keep = np.zeros((BH, N, N), dtype=np.uint8)
+    _load().ref_dropout_mask(BH, N, seed, offset, dropout_threshold(rate),
+                             keep.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+    return keep
+
+
+def ref_fwd_dropout(q, k, v, scale: float, causal: bool, rate: float, seed: int, offset: int):
+    """O [B,H,N,d] and LSE [B,H,N] in fp64 with dropout on the attention probabilities."""
+    B, H, N, d = _shape4(q)
+    qq, kk, vv = _f64(q), _f64(k), _f64(v)
+    o = np.zeros((B, H, N, d)); lse = np.zeros((B, H, N))
+    rc = _load().ref_attn_fwd_dropout(_ptr(qq), _ptr(kk), _ptr(vv), _ptr(o), _ptr(lse), B * H, N, d, float(scale),
+                                      int(bool(causal)), seed, offset, dropout_threshold(rate))
+    if rc != 0:
+        raise MemoryError("ref_attn_fwd_dropout")
+    return o, lse
+
+
+def ref_bwd_dropout(q, k, v, do, scale: float, causal: bool, rate: float, seed: int, offset: int):
+    """dQ, dK, dV [B,H,N,d] in fp64 with dropout on the attention probabilities."""
+    B, H, N, d = _shape4(q)
+    qq, kk, vv, gg = _f64(q), _f64(k), _f64(v), _f64(do)
+    dq, dk, dv = (np.zeros((B, H, N, d)) for _ in range(3))
+    rc = _load().ref_attn_bwd_dropout(_ptr(qq), _ptr(kk), _ptr(vv), _ptr(gg), _ptr(dq), _ptr(dk), _ptr(dv),
+                                      B * H, N, d, float(scale), int(bool(causal)), seed, offset,
+                                      dropout_threshold(rate))
+    if rc != 0:
+        raise MemoryError("ref_attn_bwd_dropout")
+    return dq, dk, dv
