@@ -111,6 +111,49 @@ int fa_fwd_residual(const void *q, const void *k, const void *v, void *o,
                     float scale, int causal, void *stream);
 
 /*
+ * Forward pass with dropout on the attention probabilities (the fused dropout
+ * the FlashAttention pages count among the method's largest speed-ups): the
+ * same arguments as fa_fwd_residual (o_lo may be NULL), plus
+ *   rate    dropout probability, 0 <= rate < 1 (FA_ERR_INVALID_ARG otherwise);
+ *   seed    64-bit key of the Philox4x32-10 generator (Salmon et al., SC 2011);
+ *   offset  counter word 3 (e.g. the training step): a new mask per value.
+ * Mask: for head bh = b*H + h, query row i and key j, the generator's counter is
+ * (i, j >> 3, bh, offset) and its key (seed & 0xffffffff, seed >> 32); the
+ * 16-bit draw of key j is half (j & 1) of output word ((j & 7) >> 1); key j is
+ * kept for row i iff the draw is >= T = floor(rate * 65536).  Then
+ *   O_i = sum_j P_ij * keep_ij * 65536/(65536 - T) * V_j
+ * with P = softmax(scale * Q K^T [+ causal mask]); lse is that of P, without
+ * dropout.  The mask is never stored: fa_bwd_dropout regenerates it.
+ */
+int fa_fwd_dropout(const void *q, const void *k, const void *v, void *o,
+                   void *o_lo, float *lse, int B, int H, int N, int d,
+                   float scale, int causal, float rate, unsigned long long seed,
+                   unsigned int offset, void *stream);
+
+/*
+ * Backward pass of fa_fwd_dropout, given the same rate, seed and offset (and
+ * that call's o, o_lo, lse): dV = (P o Z)^T dO, dP = Z o (dO V^T),
+ * dS = P o (dP - D) with D_i = rowsum(dO_i o O_i), dQ = scale dS K,
+ * dK = scale dS^T Q, where Z = keep * 65536/(65536 - T).  Workspace, layout and
+ * errors as fa_bwd_ex (without events).
+ */
+int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o,
+                   const void *o_lo, const void *dO, const float *lse, void *dq,
+                   void *dk, void *dv, int B, int H, int N, int d, float scale,
+                   int causal, float rate, unsigned long long seed,
+                   unsigned int offset, void *workspace, size_t workspace_bytes,
+                   void *stream);
+
+/*
+ * The dropout mask itself, for inspection and tests: mask [B,H,N,N] uint8
+ * (device, caller-owned, row-major over keys) receives keep_ij in {0, 1} as
+ * defined for fa_fwd_dropout.  This writes N*N bytes per head, the O(N^2)
+ * object the fused kernels never materialise.
+ */
+int fa_dropout_mask(int B, int H, int N, float rate, unsigned long long seed,
+                    unsigned int offset, void *mask, void *stream);
+
+/*
  * Backward pass with the optional extras:
  *   o_lo    NULL, or the residual written by fa_fwd_residual (then
  *           D_i = rowsum(dO o (o + o_lo)) instead of rowsum(dO o o));

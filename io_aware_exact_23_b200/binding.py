@@ -51,6 +51,14 @@ def lib() -> ctypes.CDLL:
         L.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp,
                                 ctypes.POINTER(vp)]
         L.fa_bwd_ex.restype = i
+        u64, u32 = ctypes.c_ulonglong, ctypes.c_uint
+        L.fa_fwd_dropout.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, f, u64, u32, vp]
+        L.fa_fwd_dropout.restype = i
+        L.fa_bwd_dropout.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, f, u64, u32, vp, sz,
+                                     vp]
+        L.fa_bwd_dropout.restype = i
+        L.fa_dropout_mask.argtypes = [i, i, i, f, u64, u32, vp, vp]
+        L.fa_dropout_mask.restype = i
         L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
         L.fa_bwd_noalloc.restype = i
         L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
@@ -200,3 +208,48 @@ class Attention:
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, self.scale, self.causal, ws, o_lo=o_lo)
         return dq, dk, dv
+
+
+def fa_fwd_dropout(q, k, v, o, lse, scale: float, causal: bool, rate: float, seed: int, offset: int = 0,
+                   stream=None, o_lo=None) -> None:
+    """Forward with dropout on the attention probabilities (``fa_fwd_dropout``)."""
+    B, H, N, d = q.shape
+    for nm, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _check(t, nm, torch.bfloat16, (B, H, N, d))
+    _check(lse, "lse", torch.float32, (B, H, N))
+    if o_lo is not None:
+        _check(o_lo, "o_lo", torch.bfloat16, (B, H, N, d))
+    rc = lib().fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              o_lo.data_ptr() if o_lo is not None else None, lse.data_ptr(), B, H, N, d,
+                              float(scale), int(bool(causal)), float(rate), int(seed) & (2**64 - 1),
+                              int(offset) & 0xFFFFFFFF, _stream_handle(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_dropout")
+
+
+def fa_bwd_dropout(q, k, v, o, dO, lse, dq, dk, dv, scale: float, causal: bool, rate: float, seed: int,
+                   workspace, offset: int = 0, stream=None, o_lo=None) -> None:
+    """Backward of ``fa_fwd_dropout`` (the mask is regenerated from rate, seed and offset)."""
+    B, H, N, d = q.shape
+    for nm, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dO", dO), ("dq", dq), ("dk", dk), ("dv", dv)):
+        _check(t, nm, torch.bfloat16, (B, H, N, d))
+    _check(lse, "lse", torch.float32, (B, H, N))
+    _check(workspace, "workspace", torch.uint8)
+    if o_lo is not None:
+        _check(o_lo, "o_lo", torch.bfloat16, (B, H, N, d))
+    rc = lib().fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              o_lo.data_ptr() if o_lo is not None else None, dO.data_ptr(), lse.data_ptr(),
+                              dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, float(scale),
+                              int(bool(causal)), float(rate), int(seed) & (2**64 - 1), int(offset) & 0xFFFFFFFF,
+                              workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_bwd_dropout")
+
+
+def fa_dropout_mask(B: int, H: int, N: int, rate: float, seed: int, offset: int, mask, stream=None) -> None:
+    """keep[b, h, i, j] in {0, 1} into the uint8 CUDA tensor ``mask`` [B,H,N,N]."""
+    _check(mask, "mask", torch.uint8, (B, H, N, N))
+    rc = lib().fa_dropout_mask(B, H, N, float(rate), int(seed) & (2**64 - 1), int(offset) & 0xFFFFFFFF,
+                               mask.data_ptr(), _stream_handle(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_dropout_mask")

@@ -1,0 +1,63 @@
+// dropout.cuh -- the counter-based generator behind fused dropout on the
+// attention probabilities (forward: P before the PV product; backward: the same
+// mask regenerated, never stored).
+//
+// Generator: Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random
+// numbers: as easy as 1, 2, 3", SC 2011): ten rounds over a 128-bit counter
+// with a 64-bit key; each round multiplies counter words 0 and 2 by the round
+// multipliers, combines the 64-bit products' halves with words 1 and 3 and the
+// key, and advances the key by the two Weyl increments.
+//
+// Mask layout: for head bh, query row i and key j the counter is
+// (i, j >> 3, bh, offset), the key is the 64-bit seed (low word, high word);
+// the 16-bit draw of key j is half (j & 1) of output word ((j & 7) >> 1), and
+// the key is kept iff the draw is >= T = floor(rate * 65536).  Kept entries
+// are scaled by 65536 / (65536 - T).
+#pragma once
+
+#include <cstdint>
+
+namespace fa {
+
+struct DropoutParams {
+  uint32_t T;        // drop a key when its 16-bit draw is below T
+  uint32_t seed_lo;  // Philox key
+  uint32_t seed_hi;
+  uint32_t offset;   // counter word 3 (e.g. the training step)
+  float inv_keep;    // 65536 / (65536 - T)
+};
+
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int round = 0; round < 10; ++round) {
+    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return c;
+}
+
+// The four output words for query row i and keys 8*jblk .. 8*jblk+7.
+__device__ __forceinline__ uint4 dropout_words(const DropoutParams &dp, uint32_t i, uint32_t jblk, uint32_t bh) {
+  return philox4x32_10(make_uint4(i, jblk, bh, dp.offset), dp.seed_lo, dp.seed_hi);
+}
+
+// Keep bits of keys 8*jblk + t (bit t), t = 0..7.
+__device__ __forceinline__ uint32_t dropout_keep8(const DropoutParams &dp, uint32_t i, uint32_t jblk, uint32_t bh) {
+  const uint4 w = dropout_words(dp, i, jblk, bh);
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  uint32_t bits = 0;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) bits |= static_cast<uint32_t>(((ws[t >> 1] >> (16 * (t & 1))) & 0xFFFFu) >= dp.T) << t;
+  return bits;
+}
+
+// bf16-pair mask for a packed word whose low half is key 2c and high half key 2c+1.
+__device__ __forceinline__ uint32_t keep_pair_mask(uint64_t keep, int c) {
+  const uint32_t b = static_cast<uint32_t>(keep >> (2 * c)) & 3u;
+  return ((b & 1u) ? 0x0000FFFFu : 0u) | ((b & 2u) ? 0xFFFF0000u : 0u);
+}
+
+}  // namespace fa

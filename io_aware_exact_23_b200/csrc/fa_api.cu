@@ -89,6 +89,26 @@ int check_shape(int B, int H, int N, int d, float scale, int causal) {
   return FA_OK;
 }
 
+template <int D, bool CAUSAL, bool DROPOUT>
+cudaError_t fwd_set_attribute() {
+  return cudaFuncSetAttribute(fa::fa_fwd_kernel<D, CAUSAL, DROPOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              fa::FwdCfg<D>::kSmemBytes);
+}
+
+// Dropout rate -> the generator's threshold and the kept entries' scale.
+// Returns false for a rate outside [0, 1).
+bool dropout_params(float rate, unsigned long long seed, unsigned int offset, fa::DropoutParams *dp) {
+  if (!std::isfinite(rate) || rate < 0.f || rate >= 1.f) return false;
+  const double t = std::floor(static_cast<double>(rate) * 65536.0);
+  if (t >= 65536.0) return false;
+  dp->T = static_cast<uint32_t>(t);
+  dp->seed_lo = static_cast<uint32_t>(seed & 0xffffffffull);
+  dp->seed_hi = static_cast<uint32_t>(seed >> 32);
+  dp->offset = offset;
+  dp->inv_keep = static_cast<float>(65536.0 / (65536.0 - t));
+  return true;
+}
+
 // Lazily set up the current device: compute capability check, SM count and
 // the status block.  Returns a status code.
 int device_state(DeviceState **out, int *dev_out) {
@@ -125,22 +145,14 @@ int device_state(DeviceState **out, int *dev_out) {
   }
   if (!s.attrs_set) {
     cudaError_t e = cudaSuccess;
-    e = (e == cudaSuccess) ? cudaFuncSetAttribute(fa::fa_fwd_kernel<64, false>,
-                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  fa::FwdCfg<64>::kSmemBytes)
-                           : e;
-    e = (e == cudaSuccess) ? cudaFuncSetAttribute(fa::fa_fwd_kernel<64, true>,
-                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  fa::FwdCfg<64>::kSmemBytes)
-                           : e;
-    e = (e == cudaSuccess) ? cudaFuncSetAttribute(fa::fa_fwd_kernel<128, false>,
-                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  fa::FwdCfg<128>::kSmemBytes)
-                           : e;
-    e = (e == cudaSuccess) ? cudaFuncSetAttribute(fa::fa_fwd_kernel<128, true>,
-                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  fa::FwdCfg<128>::kSmemBytes)
-                           : e;
+    e = (e == cudaSuccess) ? fwd_set_attribute<64, false, false>() : e;
+    e = (e == cudaSuccess) ? fwd_set_attribute<64, true, false>() : e;
+    e = (e == cudaSuccess) ? fwd_set_attribute<128, false, false>() : e;
+    e = (e == cudaSuccess) ? fwd_set_attribute<128, true, false>() : e;
+    e = (e == cudaSuccess) ? fwd_set_attribute<64, false, true>() : e;
+    e = (e == cudaSuccess) ? fwd_set_attribute<64, true, true>() : e;
+    e = (e == cudaSuccess) ? fwd_set_attribute<128, false, true>() : e;
+    e = (e == cudaSuccess) ? fwd_set_attribute<128, true, true>() : e;
     e = (e == cudaSuccess) ? fa::bwd_set_attributes() : e;
     if (e != cudaSuccess) {
       cudaGetLastError();
@@ -153,16 +165,49 @@ int device_state(DeviceState **out, int *dev_out) {
   return FA_OK;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool DROPOUT>
 cudaError_t launch_fwd(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v, const CUtensorMap &o,
                        const CUtensorMap &olo, const fa::FwdParams &p, cudaStream_t stream) {
   const dim3 grid(static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.n_qpairs));
-  fa::fa_fwd_kernel<D, CAUSAL><<<grid, fa::FwdCfg<D>::kThreads, fa::FwdCfg<D>::kSmemBytes, stream>>>(q, k, v, o, olo,
-                                                                                                      p);
+  fa::fa_fwd_kernel<D, CAUSAL, DROPOUT>
+      <<<grid, fa::FwdCfg<D>::kThreads, fa::FwdCfg<D>::kSmemBytes, stream>>>(q, k, v, o, olo, p);
   return cudaGetLastError();
 }
 
+template <bool DROPOUT>
+cudaError_t launch_fwd_any(int d, int causal, const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
+                           const CUtensorMap &o, const CUtensorMap &olo, const fa::FwdParams &p, cudaStream_t s) {
+  if (d == 64)
+    return causal ? launch_fwd<64, true, DROPOUT>(q, k, v, o, olo, p, s)
+                  : launch_fwd<64, false, DROPOUT>(q, k, v, o, olo, p, s);
+  return causal ? launch_fwd<128, true, DROPOUT>(q, k, v, o, olo, p, s)
+                : launch_fwd<128, false, DROPOUT>(q, k, v, o, olo, p, s);
+}
+
+// Dropout mask writer: one thread per (head, query row, 8-key block).
+__global__ void fa_dropout_mask_kernel(uint8_t *mask, long BH, int N, fa::DropoutParams dp) {
+  const long nblk = (N + 7) / 8;
+  const long total = BH * N * nblk;
+  for (long t = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<long>(gridDim.x) * blockDim.x) {
+    const long jb = t % nblk, row = t / nblk;
+    const long i = row % N, bh = row / N;
+    const uint32_t bits = fa::dropout_keep8(dp, static_cast<uint32_t>(i), static_cast<uint32_t>(jb),
+                                            static_cast<uint32_t>(bh));
+    uint8_t *out = mask + row * N + jb * 8;
+    for (int u = 0; u < 8 && jb * 8 + u < N; ++u) out[u] = static_cast<uint8_t>((bits >> u) & 1u);
+  }
+}
+
 }  // namespace
+
+// The shared bodies of the plain, residual and dropout entry points.
+static int fwd_common(const void *q, const void *k, const void *v, void *o, void *o_lo, float *lse, int B, int H,
+                      int N, int d, float scale, int causal, const fa::DropoutParams *drop, void *stream);
+static int bwd_common(const void *q, const void *k, const void *v, const void *o, const void *o_lo, const void *dO,
+                      const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale,
+                      int causal, void *workspace, size_t workspace_bytes, void *stream, void *const *events,
+                      const fa::DropoutParams *drop);
 
 extern "C" {
 
@@ -185,6 +230,37 @@ const char *fa_status_string(int status) {
 
 int fa_fwd_residual(const void *q, const void *k, const void *v, void *o, void *o_lo, float *lse, int B, int H,
                     int N, int d, float scale, int causal, void *stream) {
+  return fwd_common(q, k, v, o, o_lo, lse, B, H, N, d, scale, causal, nullptr, stream);
+}
+
+int fa_fwd_dropout(const void *q, const void *k, const void *v, void *o, void *o_lo, float *lse, int B, int H, int N,
+                   int d, float scale, int causal, float rate, unsigned long long seed, unsigned int offset,
+                   void *stream) {
+  fa::DropoutParams dp;
+  if (!dropout_params(rate, seed, offset, &dp)) return FA_ERR_INVALID_ARG;
+  return fwd_common(q, k, v, o, o_lo, lse, B, H, N, d, scale, causal, &dp, stream);
+}
+
+int fa_dropout_mask(int B, int H, int N, float rate, unsigned long long seed, unsigned int offset, void *mask,
+                    void *stream) {
+  if (!mask) return FA_ERR_INVALID_ARG;
+  int st = check_shape(B, H, N, 64, 1.f, 0);
+  if (st != FA_OK) return st;
+  fa::DropoutParams dp;
+  if (!dropout_params(rate, seed, offset, &dp)) return FA_ERR_INVALID_ARG;
+  DeviceState *ds = nullptr;
+  st = device_state(&ds, nullptr);
+  if (st != FA_OK) return st;
+  const long BH = static_cast<long>(B) * H;
+  fa_dropout_mask_kernel<<<ds->num_sms * 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint8_t *>(mask), BH, N, dp);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // extern "C"
+
+static int fwd_common(const void *q, const void *k, const void *v, void *o, void *o_lo, float *lse, int B, int H,
+                      int N, int d, float scale, int causal, const fa::DropoutParams *drop, void *stream) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   int st = check_shape(B, H, N, d, scale, causal);
   if (st != FA_OK) return st;
@@ -209,15 +285,15 @@ int fa_fwd_residual(const void *q, const void *k, const void *v, void *o, void *
   p.BH = BH;
   p.n_qpairs = (N + 255) / 256;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.drop = drop ? *drop : fa::DropoutParams{0u, 0u, 0u, 0u, 1.f};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e;
-  if (d == 64)
-    e = causal ? launch_fwd<64, true>(tq, tk, tv, to, tolo, p, s) : launch_fwd<64, false>(tq, tk, tv, to, tolo, p, s);
-  else
-    e = causal ? launch_fwd<128, true>(tq, tk, tv, to, tolo, p, s)
-               : launch_fwd<128, false>(tq, tk, tv, to, tolo, p, s);
+  const cudaError_t e = drop ? launch_fwd_any<true>(d, causal, tq, tk, tv, to, tolo, p, s)
+                             : launch_fwd_any<false>(d, causal, tq, tk, tv, to, tolo, p, s);
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
+
+extern "C" {
+
 
 int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N, int d,
            float scale, int causal, void *stream) {
@@ -232,6 +308,26 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
 int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o, const void *o_lo, const void *dO,
               const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale, int causal,
               void *workspace, size_t workspace_bytes, void *stream, void *const *events) {
+  return bwd_common(q, k, v, o, o_lo, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes,
+                    stream, events, nullptr);
+}
+
+int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o, const void *o_lo, const void *dO,
+                   const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale,
+                   int causal, float rate, unsigned long long seed, unsigned int offset, void *workspace,
+                   size_t workspace_bytes, void *stream) {
+  fa::DropoutParams dp;
+  if (!dropout_params(rate, seed, offset, &dp)) return FA_ERR_INVALID_ARG;
+  return bwd_common(q, k, v, o, o_lo, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes,
+                    stream, nullptr, &dp);
+}
+
+}  // extern "C"
+
+static int bwd_common(const void *q, const void *k, const void *v, const void *o, const void *o_lo, const void *dO,
+                      const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale,
+                      int causal, void *workspace, size_t workspace_bytes, void *stream, void *const *events,
+                      const fa::DropoutParams *drop) {
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   int st = check_shape(B, H, N, d, scale, causal);
   if (st != FA_OK) return st;
@@ -255,6 +351,7 @@ int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o, const 
   L.seq = next_seq();
   L.num_sms = ds->num_sms;
   L.events = reinterpret_cast<cudaEvent_t const *>(events);
+  L.drop = drop;
   CUtensorMap maps[7];
   if (encode_bf16(&maps[0], q, d, N, BH) || encode_bf16(&maps[1], k, d, N, BH) ||
       encode_bf16(&maps[2], v, d, N, BH) || encode_bf16(&maps[3], dO, d, N, BH) ||
@@ -264,6 +361,9 @@ int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o, const 
   cudaError_t e = fa::bwd_launch(L, maps, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
+
+extern "C" {
+
 
 int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dO, const float *lse, void *dq,
            void *dk, void *dv, int B, int H, int N, int d, float scale, int causal, void *workspace,

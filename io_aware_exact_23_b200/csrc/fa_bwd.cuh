@@ -45,6 +45,7 @@
 // key tiles add into them.
 #pragma once
 
+#include "dropout.cuh"
 #include "ptx.cuh"
 
 namespace fa {
@@ -60,6 +61,7 @@ struct BwdParams {
   int BH;
   float scale_log2;
   float scale;
+  DropoutParams drop;  // read only by the DROPOUT instantiations
 };
 
 constexpr int kHeadChunk = 8;  // heads whose CTAs are scheduled together
@@ -196,7 +198,7 @@ __global__ void __launch_bounds__(256) fa_dq_convert_kernel(const float *__restr
 }
 
 // ------------------------------------------------------------ main kernel
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool DROPOUT = false>
 __global__ void __launch_bounds__(448, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -460,6 +462,30 @@ __global__ void __launch_bounds__(448, 1)
       if (!ok) break;
       tc_fence_after();
       if (threadIdx.x == 0) FA_TRACE(16 + it * 8 + 4);
+      // Dropout: keep bit cc for query i*128 + 64w + cc and this thread's key.
+      // The generator's counter blocks run along keys, so the warp draws the
+      // 64 x 32 block together (eight calls per lane) and transposes it through
+      // its own rows of the dS tile, free once the previous tile's dK / dQ are done.
+      uint64_t keep = ~0ull;
+      if constexpr (DROPOUT) {
+        if (it > 0) ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, (it - 1) & 1, kBTagDkqDone));
+        if (!ok) break;
+        const uint32_t slot = smem_u32(sdS) + w * 16384 + (warp & 3) * 4096;  // [64 queries][32 keys] u16
+        const int b = lane & 3;
+        const uint32_t jblk = static_cast<uint32_t>(j * 128 + (warp & 3) * 32) / 8 + b;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int ii = (lane >> 2) + 8 * t;
+          const uint4 wv = dropout_words(p.drop, i * 128 + 64 * w + ii, jblk, bh);
+          st_shared_v4(slot + (ii * 32 + 8 * b) * 2, wv.x, wv.y, wv.z, wv.w);
+        }
+        __syncwarp();
+        const uint16_t *draws = reinterpret_cast<const uint16_t *>(sdS + w * 16384 + (warp & 3) * 4096);
+        keep = 0;
+#pragma unroll
+        for (int ii = 0; ii < 64; ++ii) keep |= static_cast<uint64_t>(draws[ii * 32 + lane] >= p.drop.T) << ii;
+        __syncwarp();
+      }
       uint32_t sv[64];
       tmem_ld32(tS + 64 * w, sv);
       tmem_ld32(tS + 64 * w + 32, sv + 32);
@@ -474,9 +500,11 @@ __global__ void __launch_bounds__(448, 1)
         for (int cc = 0; cc < 64; ++cc)
           if (64 * w + cc < r) pf[cc] = 0.f;
       }
+      // Z = keep / (keep probability): dV takes (P o Z)^T, dS the dP o Z.
+      auto zval = [&](int cc) { return DROPOUT ? (((keep >> cc) & 1ull) ? p.drop.inv_keep : 0.f) : 1.f; };
       uint32_t pk[32];
 #pragma unroll
-      for (int t = 0; t < 32; ++t) pk[t] = pack_bf16(pf[2 * t], pf[2 * t + 1]);
+      for (int t = 0; t < 32; ++t) pk[t] = pack_bf16(pf[2 * t] * zval(2 * t), pf[2 * t + 1] * zval(2 * t + 1));
       tmem_st32(tS + 64 * w, pk);  // inside the columns this warp has read
       tmem_wait_st();
       tc_fence_before();
@@ -499,8 +527,8 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
           const int c0 = 32 * ch + 2 * t;
-          const float d0 = pf[c0] * (__uint_as_float(dp[2 * t]) - Dv[c0]);
-          const float d1 = pf[c0 + 1] * (__uint_as_float(dp[2 * t + 1]) - Dv[c0 + 1]);
+          const float d0 = pf[c0] * (__uint_as_float(dp[2 * t]) * zval(c0) - Dv[c0]);
+          const float d1 = pf[c0 + 1] * (__uint_as_float(dp[2 * t + 1]) * zval(c0 + 1) - Dv[c0 + 1]);
           dsk[t] = pack_bf16(d0, d1);
         }
 #pragma unroll
@@ -648,28 +676,30 @@ struct BwdLaunch {
   int seq;
   int num_sms;
   cudaEvent_t const *events = nullptr;  // optional: 4 events recorded around the stages
+  const DropoutParams *drop = nullptr;  // dropout on the probabilities, or none
 };
 
-inline cudaError_t bwd_set_attributes() {
-  cudaError_t e = cudaFuncSetAttribute(fa_bwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       BwdCfg<64>::kSmemBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fa_bwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             BwdCfg<64>::kSmemBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fa_bwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             BwdCfg<128>::kSmemBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fa_bwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             BwdCfg<128>::kSmemBytes);
-  return e;
+template <int D, bool CAUSAL, bool DROPOUT>
+inline cudaError_t bwd_set_attribute() {
+  return cudaFuncSetAttribute(fa_bwd_kernel<D, CAUSAL, DROPOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              BwdCfg<D>::kSmemBytes);
 }
 
-template <int D, bool CAUSAL>
+inline cudaError_t bwd_set_attributes() {
+  const cudaError_t es[8] = {bwd_set_attribute<64, false, false>(), bwd_set_attribute<64, true, false>(),
+                             bwd_set_attribute<128, false, false>(), bwd_set_attribute<128, true, false>(),
+                             bwd_set_attribute<64, false, true>(), bwd_set_attribute<64, true, true>(),
+                             bwd_set_attribute<128, false, true>(), bwd_set_attribute<128, true, true>()};
+  for (cudaError_t e : es)
+    if (e != cudaSuccess) return e;
+  return cudaSuccess;
+}
+
+template <int D, bool CAUSAL, bool DROPOUT>
 inline void bwd_main_launch(const CUtensorMap *m, const BwdParams &p, int nkv, cudaStream_t s) {
   const dim3 grid(static_cast<unsigned>(p.BH) * static_cast<unsigned>(nkv));
-  fa_bwd_kernel<D, CAUSAL><<<grid, BwdCfg<D>::kThreads, BwdCfg<D>::kSmemBytes, s>>>(m[0], m[1], m[2], m[3], m[4],
-                                                                                      m[5], m[6], p);
+  fa_bwd_kernel<D, CAUSAL, DROPOUT><<<grid, BwdCfg<D>::kThreads, BwdCfg<D>::kSmemBytes, s>>>(m[0], m[1], m[2], m[3],
+                                                                                               m[4], m[5], m[6], p);
 }
 
 // maps: Q, K, V, dO, dK, dV (bf16, 3-D, 64-feature boxes), dQ accumulator
@@ -696,6 +726,7 @@ inline cudaError_t bwd_launch(const BwdLaunch &L, const CUtensorMap *maps, cudaS
   if (e != cudaSuccess) return e;
   if (L.events && (e = cudaEventRecord(L.events[1], s)) != cudaSuccess) return e;
   BwdParams p;
+  p.drop = DropoutParams{0u, 0u, 0u, 0u, 1.f};
   p.ws_lse2 = ws_lse2;
   p.ws_D = ws_D;
   p.ws_dq = ws_dq;
@@ -707,10 +738,21 @@ inline cudaError_t bwd_launch(const BwdLaunch &L, const CUtensorMap *maps, cudaS
   p.scale_log2 = L.scale * 1.4426950408889634f;
   p.scale = L.scale;
   const int nkv = Npad / 128;
-  if (L.d == 64)
-    L.causal ? bwd_main_launch<64, true>(maps, p, nkv, s) : bwd_main_launch<64, false>(maps, p, nkv, s);
-  else
-    L.causal ? bwd_main_launch<128, true>(maps, p, nkv, s) : bwd_main_launch<128, false>(maps, p, nkv, s);
+  if (L.drop) p.drop = *L.drop;
+  if (L.drop) {
+    if (L.d == 64)
+      L.causal ? bwd_main_launch<64, true, true>(maps, p, nkv, s) : bwd_main_launch<64, false, true>(maps, p, nkv, s);
+    else
+      L.causal ? bwd_main_launch<128, true, true>(maps, p, nkv, s)
+               : bwd_main_launch<128, false, true>(maps, p, nkv, s);
+  } else {
+    if (L.d == 64)
+      L.causal ? bwd_main_launch<64, true, false>(maps, p, nkv, s)
+               : bwd_main_launch<64, false, false>(maps, p, nkv, s);
+    else
+      L.causal ? bwd_main_launch<128, true, false>(maps, p, nkv, s)
+               : bwd_main_launch<128, false, false>(maps, p, nkv, s);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (L.events && (e = cudaEventRecord(L.events[2], s)) != cudaSuccess) return e;

@@ -43,6 +43,7 @@
 // delays the MMA issue more than the MUFU queue does.
 #pragma once
 
+#include "dropout.cuh"
 #include "ptx.cuh"
 
 namespace fa {
@@ -56,6 +57,7 @@ struct FwdParams {
   int BH;
   int n_qpairs;      // ceil(N / 256)
   float scale_log2;  // scale * log2(e)
+  DropoutParams drop;  // read only by the DROPOUT instantiations
 };
 
 template <int D>
@@ -97,7 +99,7 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool DROPOUT = false>
 __global__ void __launch_bounds__(352, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -319,6 +321,16 @@ __global__ void __launch_bounds__(352, 1)
           for (int cc = 0; cc < 64; ++cc)
             if (cc >= nv) s[cc] = __float_as_uint(-INFINITY);
         }
+        // Dropout: keep bit cc for key j*128 + 64h + cc of query row qt*128 + r,
+        // eight keys per generator call (the counter's key block).
+        uint64_t keep = ~0ull;
+        if constexpr (DROPOUT) {
+          keep = 0;
+          const uint32_t jb0 = static_cast<uint32_t>(j * 128 + 64 * h) >> 3;
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            keep |= static_cast<uint64_t>(dropout_keep8(p.drop, qt * 128 + r, jb0 + t, bh)) << (8 * t);
+        }
         // Half-row max as a shallow tree (eight independent chains of four).
         float mq[8];
 #pragma unroll
@@ -344,9 +356,11 @@ __global__ void __launch_bounds__(352, 1)
             f2unpack(x2, x0, x1);
             const float a = ex2(x0), b = ex2(x1);
             acc[cc & 1] = fadd2(acc[cc & 1], f2pack(a, b));
-            pk[cc] = pack_bf16(a, b);
-            racc[cc & 1] =
-                fadd2(racc[cc & 1], f2pack(__uint_as_float(pk[cc] << 16), __uint_as_float(pk[cc] & 0xFFFF0000u)));
+            const uint32_t w = pack_bf16(a, b);
+            // The sums are of P before dropout; the PV product takes the kept entries
+            // (the 1/keep-probability scale is applied to O in the epilogue).
+            pk[cc] = DROPOUT ? (w & keep_pair_mask(keep, cc)) : w;
+            racc[cc & 1] = fadd2(racc[cc & 1], f2pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
           }
           float u0, u1, u2, u3, v0, v1, v2, v3;
           f2unpack(acc[0], u0, u1);
@@ -415,7 +429,7 @@ __global__ void __launch_bounds__(352, 1)
       if (r == 0 && h == 0) FA_TRACE(4 + k);
       const float lt = l[k] + ls[((h ^ 1) * 2 + 0) * 128 + r];
       const float lrt = lr[k] + ls[((h ^ 1) * 2 + 1) * 128 + r];
-      const float inv_l = 1.f / lrt;
+      const float inv_l = (DROPOUT ? p.drop.inv_keep : 1.f) / lrt;
       const uint32_t st_o = smem_u32(sKV + (2 * k) * C::kTileBytes);
       const uint32_t st_lo = smem_u32(sKV + (2 * k + 1) * C::kTileBytes);
       const uint32_t tO = tmem + lane_off + 256 + k * D;

@@ -122,3 +122,21 @@ def test_product_path_never_imports_the_oracle():
                 txt = open(os.path.join(dirpath, fn)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, fn
                 assert "ref_attn" not in txt, fn
+
+
+def test_dropout_argument_errors(lib):
+    import ctypes as C
+    u64, u32 = C.c_ulonglong, C.c_uint
+    lib.fa_fwd_dropout.argtypes = [C.c_void_p] * 6 + [C.c_int] * 4 + [C.c_float, C.c_int, C.c_float, u64, u32,
+                                                                      C.c_void_p]
+    lib.fa_dropout_mask.argtypes = [C.c_int] * 3 + [C.c_float, u64, u32, C.c_void_p, C.c_void_p]
+
+    def fwd_d(rate, d=64):
+        return lib.fa_fwd_dropout(P, P, P, P, None, P, 1, 2, 256, d, 0.125, 0, rate, 1, 0, None)
+    assert fwd_d(-0.1) == 1 and fwd_d(1.0) == 1 and fwd_d(float("nan")) == 1
+    assert fwd_d(0.1, d=96) == 2
+    assert lib.fa_dropout_mask(1, 2, 64, 1.5, 1, 0, P, None) == 1
+    assert lib.fa_dropout_mask(1, 2, 64, 0.5, 1, 0, None, None) == 1
+    import torch
+    if not torch.cuda.is_available():
+        assert fwd_d(0.1) == 5 and lib.fa_dropout_mask(1, 2, 64, 0.5, 1, 0, P, None) == 5
