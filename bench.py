@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--cpu-budget-s", type=float, default=12.0,
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dropout", type=float, default=0.0,
+                    help="time the fused-dropout step (fa_fwd_dropout + fa_bwd_dropout) at this rate, 1 GPU")
     return ap.parse_args()
 
 
@@ -314,6 +316,65 @@ def run_vanilla(args, w):
     return 0
 
 
+def run_dropout(args, w):
+    """--dropout RATE (1 GPU): the IO-aware step with fused dropout on the probabilities."""
+    import torch
+    from io_aware_exact_23_b200 import binding as fa
+    from io_aware_exact_23_b200.inputs import make_inputs
+    dev = torch.device("cuda:0")
+    t = make_inputs(w, device=dev)
+    q, k, v, dO = t["q"], t["k"], t["v"], t["do"]
+    B, H, N, d = q.shape
+    o, o_lo = torch.empty_like(q), torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws = torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    seed = 0x5EED
+
+    def step(s_, ev=None):
+        if ev is not None:
+            ev[0].record()
+        fa.fa_fwd_dropout(q, k, v, o, lse, w.scale, w.causal, args.dropout, seed, s_, o_lo=o_lo)
+        if ev is not None:
+            ev[1].record()
+        fa.fa_bwd_dropout(q, k, v, o, dO, lse, dq, dk, dv, w.scale, w.causal, args.dropout, seed, ws, offset=s_,
+                          o_lo=o_lo)
+        if ev is not None:
+            ev[2].record()
+
+    for s_ in range(max(args.warmup, 0)):
+        step(s_)
+    K = args.steps
+    evs = [(mk(), mk(), mk()) for _ in range(K)]
+    start, end = mk(), mk()
+    torch.cuda.synchronize()
+    start.record()
+    for s_ in range(K):
+        step(args.warmup + s_, evs[s_])
+    end.record()
+    torch.cuda.synchronize()
+    if fa.fa_device_status() != 0:
+        raise SystemExit("bench.py: device status error")
+    ms = start.elapsed_time(end)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    flops = w.fwd_flops() + w.bwd_flops()
+    fwd_tf, bwd_tf = w.fwd_flops() / (fwd_ms / 1e3) / 1e12, w.bwd_flops() / (bwd_ms / 1e3) / 1e12
+    line = {"metric": METRIC, "value": flops * K / (ms / 1e3) / 1e12, "unit": UNIT, "impl": "ours", "n_gpus": 1,
+            "steps": K, "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                       "dropout": args.dropout, "l2": l2_note(w),
+                       "step": "fa_fwd_dropout + fa_bwd_dropout (a new mask per step: offset = step)"},
+            "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf, "fwd_frac_of_peak": fwd_tf / peak,
+            "bwd_frac_of_peak": bwd_tf / peak, "peak_kind": peak_kind, "gpu_launches": 4 * K}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     world, rank, local = dist_setup()
@@ -323,6 +384,8 @@ def main():
         return run_reference(args, w, world, rank)
     if args.impl == "vanilla":
         return run_vanilla(args, w)
+    if args.dropout > 0.0:
+        return run_dropout(args, w)
 
     import torch
     import torch.distributed as dist
