@@ -60,4 +60,14 @@ __device__ __forceinline__ uint32_t keep_pair_mask(uint64_t keep, int c) {
   return ((b & 1u) ? 0x0000FFFFu : 0u) | ((b & 2u) ? 0xFFFF0000u : 0u);
 }
 
+// Bit c of the keep mask, extracted afresh at each use (volatile: the compiler may
+// not carry 64 extracted values across a wait to reuse them later).
+__device__ __forceinline__ uint32_t keep_bit_fresh(uint64_t keep, int c) {
+  uint32_t bit;
+  asm volatile("{\n\t.reg .b64 t;\n\tshr.b64 t, %1, %2;\n\tcvt.u32.u64 %0, t;\n\tand.b32 %0, %0, 1;\n\t}"
+               : "=r"(bit)
+               : "l"(keep), "r"(c));
+  return bit;
+}
+
 }  // namespace fa

@@ -473,7 +473,7 @@ __global__ void __launch_bounds__(448, 1)
         const uint32_t slot = smem_u32(sdS) + w * 16384 + (warp & 3) * 4096;  // [64 queries][32 keys] u16
         const int b = lane & 3;
         const uint32_t jblk = static_cast<uint32_t>(j * 128 + (warp & 3) * 32) / 8 + b;
-#pragma unroll
+#pragma unroll 1
         for (int t = 0; t < 8; ++t) {
           const int ii = (lane >> 2) + 8 * t;
           const uint4 wv = dropout_words(p.drop, i * 128 + 64 * w + ii, jblk, bh);
@@ -527,8 +527,13 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
           const int c0 = 32 * ch + 2 * t;
-          const float d0 = pf[c0] * (__uint_as_float(dp[2 * t]) * zval(c0) - Dv[c0]);
-          const float d1 = pf[c0 + 1] * (__uint_as_float(dp[2 * t + 1]) * zval(c0 + 1) - Dv[c0 + 1]);
+          float z0 = 1.f, z1 = 1.f;
+          if constexpr (DROPOUT) {
+            z0 = keep_bit_fresh(keep, c0) ? p.drop.inv_keep : 0.f;
+            z1 = keep_bit_fresh(keep, c0 + 1) ? p.drop.inv_keep : 0.f;
+          }
+          const float d0 = pf[c0] * (__uint_as_float(dp[2 * t]) * z0 - Dv[c0]);
+          const float d1 = pf[c0 + 1] * (__uint_as_float(dp[2 * t + 1]) * z1 - Dv[c0 + 1]);
           dsk[t] = pack_bf16(d0, d1);
         }
 #pragma unroll
