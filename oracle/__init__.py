@@ -61,9 +61,9 @@ def _load():
         lib.ref_philox4x32_10.restype = None
         lib.ref_dropout_mask.argtypes = [cl, cl, u64, u32, u32, ctypes.POINTER(ctypes.c_uint8)]
         lib.ref_dropout_mask.restype = None
-        lib.ref_attn_fwd_dropout.argtypes = [D, D, D, D, D, cl, cl, cl, cd, ci, u64, u32, u32]
+        lib.ref_attn_fwd_dropout.argtypes = [D, D, D, D, D, cl, cl, cl, cd, ci, u64, u32, u32, cl]
         lib.ref_attn_fwd_dropout.restype = ci
-        lib.ref_attn_bwd_dropout.argtypes = [D, D, D, D, D, D, D, cl, cl, cl, cd, ci, u64, u32, u32]
+        lib.ref_attn_bwd_dropout.argtypes = [D, D, D, D, D, D, D, cl, cl, cl, cd, ci, u64, u32, u32, cl]
         lib.ref_attn_bwd_dropout.restype = ci
         _lib = lib
     return _lib
@@ -199,26 +199,31 @@ def dropout_mask(BH: int, N: int, seed: int, offset: int, rate: float) -> np.nda
     return keep
 
 
-def ref_fwd_dropout(q, k, v, scale: float, causal: bool, rate: float, seed: int, offset: int):
-    """O [B,H,N,d] and LSE [B,H,N] in fp64 with dropout on the attention probabilities."""
+def ref_fwd_dropout(q, k, v, scale: float, causal: bool, rate: float, seed: int, offset: int, head0: int = 0):
+    """O [B,H,N,d] and LSE [B,H,N] in fp64 with dropout on the attention probabilities.
+
+    ``head0``: global index b*H + h of the first head passed (when checking some
+    heads of a larger workload on their own)."""
     B, H, N, d = _shape4(q)
     qq, kk, vv = _f64(q), _f64(k), _f64(v)
     o = np.zeros((B, H, N, d)); lse = np.zeros((B, H, N))
     rc = _load().ref_attn_fwd_dropout(_ptr(qq), _ptr(kk), _ptr(vv), _ptr(o), _ptr(lse), B * H, N, d, float(scale),
-                                      int(bool(causal)), seed, offset, dropout_threshold(rate))
+                                      int(bool(causal)), seed, offset, dropout_threshold(rate), head0)
     if rc != 0:
         raise MemoryError("ref_attn_fwd_dropout")
     return o, lse
 
 
-def ref_bwd_dropout(q, k, v, do, scale: float, causal: bool, rate: float, seed: int, offset: int):
-    """dQ, dK, dV [B,H,N,d] in fp64 with dropout on the attention probabilities."""
+def ref_bwd_dropout(q, k, v, do, scale: float, causal: bool, rate: float, seed: int, offset: int,
+                    head0: int = 0):
+    """dQ, dK, dV [B,H,N,d] in fp64 with dropout on the attention probabilities (``head0``
+    as for ``ref_fwd_dropout``)."""
     B, H, N, d = _shape4(q)
     qq, kk, vv, gg = _f64(q), _f64(k), _f64(v), _f64(do)
     dq, dk, dv = (np.zeros((B, H, N, d)) for _ in range(3))
     rc = _load().ref_attn_bwd_dropout(_ptr(qq), _ptr(kk), _ptr(vv), _ptr(gg), _ptr(dq), _ptr(dk), _ptr(dv),
                                       B * H, N, d, float(scale), int(bool(causal)), seed, offset,
-                                      dropout_threshold(rate))
+                                      dropout_threshold(rate), head0)
     if rc != 0:
         raise MemoryError("ref_attn_bwd_dropout")
     return dq, dk, dv

@@ -121,8 +121,11 @@ static double zval(uint64_t seed, uint32_t offset, uint32_t T, long bh, long i, 
     return draw16(seed, offset, bh, i, j) >= T ? 65536.0 / (65536.0 - (double)T) : 0.0;
 }
 
+/* bh0: global head index of the first head passed (the mask's counter uses b*H + h), so
+   that single heads of a large workload can be checked on their own. */
 int ref_attn_fwd_dropout(const double *Q, const double *K, const double *V, double *O, double *LSE, long BH,
-                         long N, long d, double scale, int causal, uint64_t seed, uint32_t offset, uint32_t T)
+                         long N, long d, double scale, int causal, uint64_t seed, uint32_t offset, uint32_t T,
+                         long bh0)
 {
     double *p = (double *)malloc(sizeof(double) * (size_t)N);
     if (!p)
@@ -136,7 +139,7 @@ int ref_attn_fwd_dropout(const double *Q, const double *K, const double *V, doub
             for (long c = 0; c < d; ++c)
                 o[c] = 0.0;
             for (long j = 0; j < N; ++j) {
-                const double w = p[j] * zval(seed, offset, T, bh, i, j);
+                const double w = p[j] * zval(seed, offset, T, bh0 + bh, i, j);
                 if (w == 0.0)
                     continue;
                 for (long c = 0; c < d; ++c)
@@ -151,7 +154,7 @@ int ref_attn_fwd_dropout(const double *Q, const double *K, const double *V, doub
 
 int ref_attn_bwd_dropout(const double *Q, const double *K, const double *V, const double *dO, double *dQ,
                          double *dK, double *dV, long BH, long N, long d, double scale, int causal, uint64_t seed,
-                         uint32_t offset, uint32_t T)
+                         uint32_t offset, uint32_t T, long bh0)
 {
     double *p = (double *)malloc(sizeof(double) * (size_t)N);
     double *dp = (double *)malloc(sizeof(double) * (size_t)N);
@@ -173,7 +176,7 @@ int ref_attn_bwd_dropout(const double *Q, const double *K, const double *V, cons
             prob_row(q, k, N, d, scale, causal, i, p, &m, &l);
             double D = 0.0;
             for (long j = 0; j < N; ++j) {
-                const double z = zval(seed, offset, T, bh, i, j);
+                const double z = zval(seed, offset, T, bh0 + bh, i, j);
                 double s = 0.0;
                 for (long c = 0; c < d; ++c)
                     s += go[i * d + c] * v[j * d + c];

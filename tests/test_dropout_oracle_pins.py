@@ -163,3 +163,20 @@ def test_unbiased_over_masks():
         acc += oracle.ref_fwd_dropout(q, k, v, 0.5, False, 0.3, 5, off)[0]
     err = np.abs(acc / n - o_plain).max()
     assert err <= 0.08 * np.abs(v).max()
+
+
+def test_single_heads_match_the_whole_batch():
+    """head0 selects the mask of a head checked on its own (global index b*H + h)."""
+    B, H, N, d = 2, 3, 20, 4
+    q, k, v, do = (rnd((B, H, N, d), 50 + s) for s in range(4))
+    args = (0.6, False, 0.3, 17, 4)
+    o, lse = oracle.ref_fwd_dropout(q, k, v, *args)
+    g = oracle.ref_bwd_dropout(q, k, v, do, *args)
+    for b in range(B):
+        for h in range(H):
+            sl = lambda x: x[b:b + 1, h:h + 1]  # noqa: E731
+            o1, l1 = oracle.ref_fwd_dropout(sl(q), sl(k), sl(v), *args, head0=b * H + h)
+            assert np.array_equal(o1[0, 0], o[b, h]) and np.array_equal(l1[0, 0], lse[b, h])
+            g1 = oracle.ref_bwd_dropout(sl(q), sl(k), sl(v), sl(do), *args, head0=b * H + h)
+            for x1, x in zip(g1, g):
+                assert np.array_equal(x1[0, 0], x[b, h])
