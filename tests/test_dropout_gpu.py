@@ -96,3 +96,24 @@ def test_offset_changes_the_mask_and_seed_reproduces_it():
     torch.cuda.synchronize()
     assert torch.equal(outs[0], outs[1])
     assert not torch.equal(outs[0], outs[2])
+
+
+def test_dropout_full_size_workload():
+    """The bench's workload (B=2, H=32, N=4096, d=128, causal) with dropout 0.1 on the GPU;
+    two whole heads (every element of O, LSE, dQ, dK, dV) against the oracle."""
+    from io_aware_exact_23_b200.inputs import C3 as w
+    rate, seed, offset = 0.1, 0x5EED, 3
+    t = make_inputs(w, device="cuda")
+    o, lse, o_lo, dq, dk, dv = run_dropout(t, w, rate, seed, offset)
+    for b, h in ((0, 0), (1, 21)):
+        sl = {nm: x[b:b + 1, h:h + 1] for nm, x in t.items()}
+        head0 = b * w.H + h
+        o_ref, lse_ref = oracle.ref_fwd_dropout(sl["q"], sl["k"], sl["v"], w.scale, True, rate, seed, offset,
+                                                head0=head0)
+        strict, pre, res = o_errors(o[b:b + 1, h:h + 1], o_ref, o_lo[b:b + 1, h:h + 1])
+        assert pre <= TOL_O and res <= TOL_O, (b, h, strict, pre, res)
+        assert max_err(to64(lse[b:b + 1, h:h + 1]), lse_ref) <= TOL_LSE
+        rq, rk, rv = oracle.ref_bwd_dropout(sl["q"], sl["k"], sl["v"], sl["do"], w.scale, True, rate, seed, offset,
+                                            head0=head0)
+        check_grads({"dq": to64(dq[b:b + 1, h:h + 1]), "dk": to64(dk[b:b + 1, h:h + 1]),
+                     "dv": to64(dv[b:b + 1, h:h + 1])}, {"dq": rq, "dk": rk, "dv": rv}, f"C3 head {head0}")
