@@ -55,6 +55,9 @@ def parse_args():
     ap.add_argument("--cpu-budget-s", type=float, default=12.0,
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one JSON line per workload (tiny, C2, C3, long and the non-stress sweep points): "
+                         "forward and backward TFLOP/s, fraction of peak, peak HBM vs the N^2 score size; 1 GPU")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="time the fused-dropout step (fa_fwd_dropout + fa_bwd_dropout) at this rate, 1 GPU")
     return ap.parse_args()
@@ -375,10 +378,58 @@ def run_dropout(args, w):
     return 0
 
 
+def run_sweep(args):
+    """--sweep: fa_fwd and fa_bwd (the default entry points) timed per workload with CUDA events."""
+    import torch
+    from io_aware_exact_23_b200 import binding as fa
+    from io_aware_exact_23_b200.inputs import C2, C3, C4, TINY, make_inputs, score_matrix_bytes, sweep
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    torch.zeros(1, device=dev)  # create the context before the memory statistics are touched
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    for w in [TINY, C2, C3, C4] + [x for x in sweep() if x.qk_mult == 1.0]:
+        torch.cuda.empty_cache()
+        torch.cuda.reset_peak_memory_stats(dev)
+        t = make_inputs(w, device=dev)
+        q, k, v, dO = t["q"], t["k"], t["v"], t["do"]
+        B, H, N, d = q.shape
+        o, lse = torch.empty_like(q), torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+        ws = torch.empty(fa.fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+        reps = max(3, min(50, int(2e12 / max(w.fwd_flops(), 1.0))))
+        for _ in range(3):
+            fa.fa_fwd(q, k, v, o, lse, w.scale, w.causal)
+            fa.fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, w.scale, w.causal, ws)
+        e = [mk() for _ in range(3)]
+        e[0].record()
+        for _ in range(reps):
+            fa.fa_fwd(q, k, v, o, lse, w.scale, w.causal)
+        e[1].record()
+        for _ in range(reps):
+            fa.fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, w.scale, w.causal, ws)
+        e[2].record()
+        torch.cuda.synchronize()
+        if fa.fa_device_status() != 0:
+            raise SystemExit(f"bench.py: device status error on {w.name}")
+        fwd_ms, bwd_ms = e[0].elapsed_time(e[1]) / reps, e[1].elapsed_time(e[2]) / reps
+        fwd_tf, bwd_tf = w.fwd_flops() / (fwd_ms / 1e3) / 1e12, w.bwd_flops() / (bwd_ms / 1e3) / 1e12
+        print(json.dumps({"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal, "reps": reps,
+                          "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+                          "fwd_frac_of_peak": fwd_tf / peak, "bwd_frac_of_peak": bwd_tf / peak,
+                          "peak_kind": peak_kind, "peak_hbm_bytes": torch.cuda.max_memory_allocated(dev),
+                          "score_matrix_bytes_bf16": score_matrix_bytes(B, H, N), "l2": l2_note(w)}), flush=True)
+        del t, q, k, v, dO, o, lse, dq, dk, dv, ws
+    return 0
+
+
 def main():
     args = parse_args()
     world, rank, local = dist_setup()
     from io_aware_exact_23_b200.inputs import CONFIGS
+    if args.sweep:
+        return run_sweep(args)
     w = CONFIGS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w, world, rank)
