@@ -16,7 +16,9 @@ Launch: ``python bench.py --gpus N --steps K --warmup W`` (one rank per GPU
 under torchrun for N > 1; every rank runs the same workload: weak scaling, no
 data-path collective).  Prints one JSON line on rank 0.
 ``--impl reference`` times the CPU fp64 oracle instead (rank 0 only);
-``--impl vanilla`` times standard attention (S and P in HBM) on one GPU.
+``--impl vanilla`` times standard attention (S and P in HBM) on one GPU;
+``--dropout RATE`` times the step with fused dropout on the probabilities;
+``--sweep`` prints one line per workload (forward and backward separately).
 """
 from __future__ import annotations
 
