@@ -18,6 +18,7 @@ data-path collective).  Prints one JSON line on rank 0.
 ``--impl reference`` times the CPU fp64 oracle instead (rank 0 only);
 ``--impl vanilla`` times standard attention (S and P in HBM) on one GPU;
 ``--dropout RATE`` times the step with fused dropout on the probabilities;
+``--deterministic`` times the step with the deterministic backward;
 ``--sweep`` prints one line per workload (forward and backward separately).
 """
 from __future__ import annotations
@@ -60,6 +61,8 @@ def parse_args():
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line per workload (tiny, C2, C3, long and the non-stress sweep points): "
                          "forward and backward TFLOP/s, fraction of peak, peak HBM vs the N^2 score size; 1 GPU")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="time the step with fa_bwd_deterministic (dQ in a fixed summation order)")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="time the fused-dropout step (fa_fwd_dropout + fa_bwd_dropout) at this rate, 1 GPU")
     return ap.parse_args()
@@ -321,8 +324,10 @@ def run_vanilla(args, w):
     return 0
 
 
-def run_dropout(args, w):
-    """--dropout RATE (1 GPU): the IO-aware step with fused dropout on the probabilities."""
+def run_variant(args, w):
+    """--dropout RATE or --deterministic (1 GPU): the IO-aware step with fused
+    dropout on the probabilities, or with the deterministic backward (dQ summed
+    over key tiles in a fixed order by its own kernel)."""
     import torch
     from io_aware_exact_23_b200 import binding as fa
     from io_aware_exact_23_b200.inputs import make_inputs
@@ -337,14 +342,22 @@ def run_dropout(args, w):
     mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     seed = 0x5EED
 
-    def step(s_, ev=None):
+    def step(s_, ev=None, plain_bwd=False):
         if ev is not None:
             ev[0].record()
-        fa.fa_fwd_dropout(q, k, v, o, lse, w.scale, w.causal, args.dropout, seed, s_, o_lo=o_lo)
+        if args.deterministic:
+            fa.fa_fwd(q, k, v, o, lse, w.scale, w.causal, o_lo=o_lo)
+        else:
+            fa.fa_fwd_dropout(q, k, v, o, lse, w.scale, w.causal, args.dropout, seed, s_, o_lo=o_lo)
         if ev is not None:
             ev[1].record()
-        fa.fa_bwd_dropout(q, k, v, o, dO, lse, dq, dk, dv, w.scale, w.causal, args.dropout, seed, ws, offset=s_,
-                          o_lo=o_lo)
+        if plain_bwd:
+            fa.fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, w.scale, w.causal, ws, o_lo=o_lo)
+        elif args.deterministic:
+            fa.fa_bwd_deterministic(q, k, v, o, dO, lse, dq, dk, dv, w.scale, w.causal, ws, o_lo=o_lo)
+        else:
+            fa.fa_bwd_dropout(q, k, v, o, dO, lse, dq, dk, dv, w.scale, w.causal, args.dropout, seed, ws,
+                              offset=s_, o_lo=o_lo)
         if ev is not None:
             ev[2].record()
 
@@ -364,6 +377,15 @@ def run_dropout(args, w):
     ms = start.elapsed_time(end)
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    extra = {}
+    if args.deterministic:
+        # context, outside the timed region: the same steps with fa_bwd (dQ added in arrival order)
+        pev = [(mk(), mk(), mk()) for _ in range(K)]
+        for s_ in range(K):
+            step(s_, pev[s_], plain_bwd=True)
+        torch.cuda.synchronize()
+        extra["bwd_ms_fa_bwd"] = statistics.mean(e[1].elapsed_time(e[2]) for e in pev)
+        extra["bwd_ms"] = bwd_ms
     peaks, peak_kind = load_peaks()
     peak = float(peaks["bf16_tflops"])
     flops = w.fwd_flops() + w.bwd_flops()
@@ -372,10 +394,11 @@ def run_dropout(args, w):
             "steps": K, "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
-                       "dropout": args.dropout, "l2": l2_note(w),
-                       "step": "fa_fwd_dropout + fa_bwd_dropout (a new mask per step: offset = step)"},
+                       "dropout": args.dropout, "deterministic": bool(args.deterministic), "l2": l2_note(w),
+                       "step": ("fa_fwd + fa_bwd_deterministic" if args.deterministic else
+                                "fa_fwd_dropout + fa_bwd_dropout (a new mask per step: offset = step)")},
             "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf, "fwd_frac_of_peak": fwd_tf / peak,
-            "bwd_frac_of_peak": bwd_tf / peak, "peak_kind": peak_kind, "gpu_launches": 4 * K}
+            "bwd_frac_of_peak": bwd_tf / peak, "peak_kind": peak_kind, "gpu_launches": 4 * K, **extra}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -437,8 +460,10 @@ def main():
         return run_reference(args, w, world, rank)
     if args.impl == "vanilla":
         return run_vanilla(args, w)
-    if args.dropout > 0.0:
-        return run_dropout(args, w)
+    if args.dropout > 0.0 and args.deterministic:
+        raise SystemExit("bench.py: --dropout and --deterministic are separate arms")
+    if args.dropout > 0.0 or args.deterministic:
+        return run_variant(args, w)
 
     import torch
     import torch.distributed as dist

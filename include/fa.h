@@ -171,6 +171,32 @@ int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o,
               void *stream, void *const *events);
 
 /*
+ * Deterministic backward pass: the same results as fa_bwd_ex (without events)
+ * within the same tolerances, and the same bits on every call with the same
+ * inputs on the same GPU model.
+ *
+ * In fa_bwd, each 128-row key tile adds its contribution dS_ij K_j to dQ_i into
+ * an fp32 accumulator as it finishes, so the order of the fp32 additions, and
+ * with it the last bits of dQ, can change from run to run.  Here dQ is
+ * computed by a separate kernel, one CTA per (head, 128-row query tile), which
+ * recomputes S_ij = Q_i K_j^T, P_ij (from LSE, as in the review's
+ * "Recomputation" section), dP_ij = dO_i V_j^T and dS_ij (the chain rule
+ * through softmax) and sums dQ_i over the key tiles in ascending j in tensor
+ * memory.  dK and dV come from the fused kernel, bit for bit as in fa_bwd.
+ * Costs about 1.6x fa_bwd's tensor-core work (the fused kernel's own dQ product
+ * is still computed and discarded).
+ *
+ * Arguments, layout, ownership and errors: as fa_bwd_ex with events = NULL
+ * (o_lo may be NULL); the workspace size is fa_bwd_workspace_bytes(B, H, N, d).
+ */
+int fa_bwd_deterministic(const void *q, const void *k, const void *v,
+                         const void *o, const void *o_lo, const void *dO,
+                         const float *lse, void *dq, void *dk, void *dv,
+                         int B, int H, int N, int d, float scale, int causal,
+                         void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+/*
  * Backward pass for callers that cannot allocate device memory.
  *
  * Some callers may not call cudaMalloc at all: code that runs where an
@@ -219,7 +245,7 @@ int fa_device_status(void *stream);
 
 /*
  * Like fa_device_status(), and also copies the failure record into info[0..3]:
- * {kernel id (1 fwd, 2 bwd, 3 bwd preprocess, 4 dQ convert), wait tag, block
+ * {kernel id (1 fwd, 2 bwd, 4 deterministic dQ), wait tag, block
  * index, launch sequence number}; zeros when there was no failure.  `info` is a
  * host pointer to 4 ints (may be NULL).
  */

@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.fa_bwd_dropout.restype = i
         L.fa_dropout_mask.argtypes = [i, i, i, f, u64, u32, vp, vp]
         L.fa_dropout_mask.restype = i
+        L.fa_bwd_deterministic.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
+        L.fa_bwd_deterministic.restype = i
         L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
         L.fa_bwd_noalloc.restype = i
         L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
@@ -157,6 +159,26 @@ def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, scale: float, causal: bool, workspac
                              handles)
     if rc != FA_OK:
         raise FaError(rc, "fa_bwd")
+
+
+def fa_bwd_deterministic(q, k, v, o, dO, lse, dq, dk, dv, scale: float, causal: bool, workspace, stream=None,
+                         o_lo=None) -> None:
+    """``fa_bwd`` with dQ summed over key tiles in a fixed order: the same bits on
+    every call (``fa_bwd_deterministic``); dK and dV are ``fa_bwd``'s."""
+    B, H, N, d = q.shape
+    for nm, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dO", dO), ("dq", dq), ("dk", dk), ("dv", dv)):
+        _check(t, nm, torch.bfloat16, (B, H, N, d))
+    _check(lse, "lse", torch.float32, (B, H, N))
+    _check(workspace, "workspace", torch.uint8)
+    if o_lo is not None:
+        _check(o_lo, "o_lo", torch.bfloat16, (B, H, N, d))
+    rc = lib().fa_bwd_deterministic(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                    o_lo.data_ptr() if o_lo is not None else None, dO.data_ptr(), lse.data_ptr(),
+                                    dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, float(scale),
+                                    int(bool(causal)), workspace.data_ptr(), workspace.numel(),
+                                    _stream_handle(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_bwd_deterministic")
 
 
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # FA_NOALLOC_SCRATCH_BYTES in include/fa.h

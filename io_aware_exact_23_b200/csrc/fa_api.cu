@@ -1,6 +1,6 @@
 // fa_api.cu -- the C ABI of libfa.so (declared in include/fa.h): argument
 // validation, TMA descriptor encoding, the per-device status block, and the
-// launches of the forward and backward kernels.
+// launches of the forward, backward and deterministic-dQ kernels.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -12,6 +12,7 @@
 
 #include "fa.h"
 #include "fa_bwd.cuh"
+#include "fa_dq.cuh"
 #include "fa_fwd.cuh"
 
 namespace {
@@ -154,6 +155,7 @@ int device_state(DeviceState **out, int *dev_out) {
     e = (e == cudaSuccess) ? fwd_set_attribute<128, false, true>() : e;
     e = (e == cudaSuccess) ? fwd_set_attribute<128, true, true>() : e;
     e = (e == cudaSuccess) ? fa::bwd_set_attributes() : e;
+    e = (e == cudaSuccess) ? fa::dq_set_attributes() : e;
     if (e != cudaSuccess) {
       cudaGetLastError();
       return FA_ERR_CUDA;
@@ -201,63 +203,8 @@ __global__ void fa_dropout_mask_kernel(uint8_t *mask, long BH, int N, fa::Dropou
 
 }  // namespace
 
-// The shared bodies of the plain, residual and dropout entry points.
-static int fwd_common(const void *q, const void *k, const void *v, void *o, void *o_lo, float *lse, int B, int H,
-                      int N, int d, float scale, int causal, const fa::DropoutParams *drop, void *stream);
-static int bwd_common(const void *q, const void *k, const void *v, const void *o, const void *o_lo, const void *dO,
-                      const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale,
-                      int causal, void *workspace, size_t workspace_bytes, void *stream, void *const *events,
-                      const fa::DropoutParams *drop);
-
-extern "C" {
-
-int fa_version(void) { return 100; }
-
-const char *fa_status_string(int status) {
-  switch (status) {
-    case FA_OK: return "FA_OK";
-    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: invalid argument";
-    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: unsupported shape or device";
-    case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED: pointer not 16-byte aligned";
-    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace missing or too small";
-    case FA_ERR_NO_DEVICE: return "FA_ERR_NO_DEVICE: no usable CUDA device";
-    case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA call or launch failed";
-    case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT: a kernel gave up on a pipeline wait";
-    case FA_ERR_DEVICE_INTERNAL: return "FA_ERR_DEVICE_INTERNAL: kernel launch environment unusable";
-    default: return "unknown fa_status";
-  }
-}
-
-int fa_fwd_residual(const void *q, const void *k, const void *v, void *o, void *o_lo, float *lse, int B, int H,
-                    int N, int d, float scale, int causal, void *stream) {
-  return fwd_common(q, k, v, o, o_lo, lse, B, H, N, d, scale, causal, nullptr, stream);
-}
-
-int fa_fwd_dropout(const void *q, const void *k, const void *v, void *o, void *o_lo, float *lse, int B, int H, int N,
-                   int d, float scale, int causal, float rate, unsigned long long seed, unsigned int offset,
-                   void *stream) {
-  fa::DropoutParams dp;
-  if (!dropout_params(rate, seed, offset, &dp)) return FA_ERR_INVALID_ARG;
-  return fwd_common(q, k, v, o, o_lo, lse, B, H, N, d, scale, causal, &dp, stream);
-}
-
-int fa_dropout_mask(int B, int H, int N, float rate, unsigned long long seed, unsigned int offset, void *mask,
-                    void *stream) {
-  if (!mask) return FA_ERR_INVALID_ARG;
-  int st = check_shape(B, H, N, 64, 1.f, 0);
-  if (st != FA_OK) return st;
-  fa::DropoutParams dp;
-  if (!dropout_params(rate, seed, offset, &dp)) return FA_ERR_INVALID_ARG;
-  DeviceState *ds = nullptr;
-  st = device_state(&ds, nullptr);
-  if (st != FA_OK) return st;
-  const long BH = static_cast<long>(B) * H;
-  fa_dropout_mask_kernel<<<ds->num_sms * 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint8_t *>(mask), BH, N, dp);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
-
-}  // extern "C"
+// ---------------------------------------------------------------------------
+// The shared bodies of the entry points: argument checks, tensor maps, launch.
 
 static int fwd_common(const void *q, const void *k, const void *v, void *o, void *o_lo, float *lse, int B, int H,
                       int N, int d, float scale, int causal, const fa::DropoutParams *drop, void *stream) {
@@ -292,42 +239,12 @@ static int fwd_common(const void *q, const void *k, const void *v, void *o, void
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-extern "C" {
-
-
-int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N, int d,
-           float scale, int causal, void *stream) {
-  return fa_fwd_residual(q, k, v, o, nullptr, lse, B, H, N, d, scale, causal, stream);
-}
-
-size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
-  if (check_shape(B, H, N, d, 1.f, 0) != FA_OK) return 0;
-  return fa::bwd_workspace_bytes(B * H, N, d);
-}
-
-int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o, const void *o_lo, const void *dO,
-              const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale, int causal,
-              void *workspace, size_t workspace_bytes, void *stream, void *const *events) {
-  return bwd_common(q, k, v, o, o_lo, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes,
-                    stream, events, nullptr);
-}
-
-int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o, const void *o_lo, const void *dO,
-                   const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale,
-                   int causal, float rate, unsigned long long seed, unsigned int offset, void *workspace,
-                   size_t workspace_bytes, void *stream) {
-  fa::DropoutParams dp;
-  if (!dropout_params(rate, seed, offset, &dp)) return FA_ERR_INVALID_ARG;
-  return bwd_common(q, k, v, o, o_lo, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes,
-                    stream, nullptr, &dp);
-}
-
-}  // extern "C"
-
+// deterministic: dQ from fa_dq_kernel (a fixed summation order over key tiles)
+// instead of the fp32 accumulator that key tiles add into as they finish.
 static int bwd_common(const void *q, const void *k, const void *v, const void *o, const void *o_lo, const void *dO,
                       const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale,
                       int causal, void *workspace, size_t workspace_bytes, void *stream, void *const *events,
-                      const fa::DropoutParams *drop) {
+                      const fa::DropoutParams *drop, bool deterministic) {
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   int st = check_shape(B, H, N, d, scale, causal);
   if (st != FA_OK) return st;
@@ -352,24 +269,105 @@ static int bwd_common(const void *q, const void *k, const void *v, const void *o
   L.num_sms = ds->num_sms;
   L.events = reinterpret_cast<cudaEvent_t const *>(events);
   L.drop = drop;
-  CUtensorMap maps[7];
+  CUtensorMap maps[7], tdq;
   if (encode_bf16(&maps[0], q, d, N, BH) || encode_bf16(&maps[1], k, d, N, BH) ||
       encode_bf16(&maps[2], v, d, N, BH) || encode_bf16(&maps[3], dO, d, N, BH) ||
       encode_bf16(&maps[4], dk, d, N, BH) || encode_bf16(&maps[5], dv, d, N, BH) ||
-      encode_3d(&maps[6], L.workspace, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, BH, 32))
+      encode_3d(&maps[6], L.workspace, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, BH, 32) ||
+      (deterministic && encode_bf16(&tdq, dq, d, N, BH)))
     return FA_ERR_CUDA;
-  cudaError_t e = fa::bwd_launch(L, maps, static_cast<cudaStream_t>(stream));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = deterministic ? fa::bwd_launch_deterministic(L, maps, tdq, s) : fa::bwd_launch(L, maps, s);
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 extern "C" {
 
+int fa_version(void) { return 100; }
+
+const char *fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: invalid argument";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: unsupported shape or device";
+    case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED: pointer not 16-byte aligned";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace missing or too small";
+    case FA_ERR_NO_DEVICE: return "FA_ERR_NO_DEVICE: no usable CUDA device";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA call or launch failed";
+    case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT: a kernel gave up on a pipeline wait";
+    case FA_ERR_DEVICE_INTERNAL: return "FA_ERR_DEVICE_INTERNAL: kernel launch environment unusable";
+    default: return "unknown fa_status";
+  }
+}
+
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N, int d,
+           float scale, int causal, void *stream) {
+  return fwd_common(q, k, v, o, nullptr, lse, B, H, N, d, scale, causal, nullptr, stream);
+}
+
+int fa_fwd_residual(const void *q, const void *k, const void *v, void *o, void *o_lo, float *lse, int B, int H,
+                    int N, int d, float scale, int causal, void *stream) {
+  return fwd_common(q, k, v, o, o_lo, lse, B, H, N, d, scale, causal, nullptr, stream);
+}
+
+int fa_fwd_dropout(const void *q, const void *k, const void *v, void *o, void *o_lo, float *lse, int B, int H, int N,
+                   int d, float scale, int causal, float rate, unsigned long long seed, unsigned int offset,
+                   void *stream) {
+  fa::DropoutParams dp;
+  if (!dropout_params(rate, seed, offset, &dp)) return FA_ERR_INVALID_ARG;
+  return fwd_common(q, k, v, o, o_lo, lse, B, H, N, d, scale, causal, &dp, stream);
+}
+
+int fa_dropout_mask(int B, int H, int N, float rate, unsigned long long seed, unsigned int offset, void *mask,
+                    void *stream) {
+  if (!mask) return FA_ERR_INVALID_ARG;
+  int st = check_shape(B, H, N, 64, 1.f, 0);
+  if (st != FA_OK) return st;
+  fa::DropoutParams dp;
+  if (!dropout_params(rate, seed, offset, &dp)) return FA_ERR_INVALID_ARG;
+  DeviceState *ds = nullptr;
+  st = device_state(&ds, nullptr);
+  if (st != FA_OK) return st;
+  const long BH = static_cast<long>(B) * H;
+  fa_dropout_mask_kernel<<<ds->num_sms * 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint8_t *>(mask), BH, N, dp);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (check_shape(B, H, N, d, 1.f, 0) != FA_OK) return 0;
+  return fa::bwd_workspace_bytes(B * H, N, d);
+}
 
 int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dO, const float *lse, void *dq,
            void *dk, void *dv, int B, int H, int N, int d, float scale, int causal, void *workspace,
            size_t workspace_bytes, void *stream) {
-  return fa_bwd_ex(q, k, v, o, nullptr, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace,
-                   workspace_bytes, stream, nullptr);
+  return bwd_common(q, k, v, o, nullptr, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace,
+                    workspace_bytes, stream, nullptr, nullptr, false);
+}
+
+int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o, const void *o_lo, const void *dO,
+              const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale, int causal,
+              void *workspace, size_t workspace_bytes, void *stream, void *const *events) {
+  return bwd_common(q, k, v, o, o_lo, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes,
+                    stream, events, nullptr, false);
+}
+
+int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o, const void *o_lo, const void *dO,
+                   const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale,
+                   int causal, float rate, unsigned long long seed, unsigned int offset, void *workspace,
+                   size_t workspace_bytes, void *stream) {
+  fa::DropoutParams dp;
+  if (!dropout_params(rate, seed, offset, &dp)) return FA_ERR_INVALID_ARG;
+  return bwd_common(q, k, v, o, o_lo, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes,
+                    stream, nullptr, &dp, false);
+}
+
+int fa_bwd_deterministic(const void *q, const void *k, const void *v, const void *o, const void *o_lo,
+                         const void *dO, const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d,
+                         float scale, int causal, void *workspace, size_t workspace_bytes, void *stream) {
+  return bwd_common(q, k, v, o, o_lo, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes,
+                    stream, nullptr, nullptr, true);
 }
 
 int fa_device_status_info(void *stream, int *info) {

@@ -140,3 +140,24 @@ def test_dropout_argument_errors(lib):
     import torch
     if not torch.cuda.is_available():
         assert fwd_d(0.1) == 5 and lib.fa_dropout_mask(1, 2, 64, 0.5, 1, 0, P, None) == 5
+
+
+@pytest.mark.parametrize("kw,code", [
+    ({"dq": None}, 1), ({"N": 0}, 1), ({"scale": 0.0}, 1), ({"causal": 3}, 1), ({"d": 80}, 2),
+    ({"ws": None}, 4), ({"ws_bytes": 16}, 4), ({"ws": ctypes.c_void_p(4104)}, 3),
+    ({"dq": ctypes.c_void_p(4098)}, 3), ({"o_lo": ctypes.c_void_p(4100)}, 3),
+])
+def test_deterministic_bwd_argument_errors(lib, kw, code):
+    args = dict(ws=P, ws_bytes=1 << 30, N=256, d=64, scale=0.125, causal=0, dq=P, o_lo=None)
+    args.update(kw)
+    rc = lib.fa_bwd_deterministic(P, P, P, P, args["o_lo"], P, P, args["dq"], P, P, 1, 2, args["N"], args["d"],
+                                  args["scale"], args["causal"], args["ws"], args["ws_bytes"], None)
+    assert rc == code
+
+
+def test_deterministic_bwd_without_a_device(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    assert lib.fa_bwd_deterministic(P, P, P, P, None, P, P, P, P, P, 1, 2, 256, 64, 0.125, 1, P, 1 << 30,
+                                    None) == 5
