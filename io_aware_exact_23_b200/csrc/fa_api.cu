@@ -283,7 +283,7 @@ static int bwd_common(const void *q, const void *k, const void *v, const void *o
 
 extern "C" {
 
-int fa_version(void) { return 100; }
+int fa_version(void) { return 200; }  // 0.2.0: fa_bwd_deterministic
 
 const char *fa_status_string(int status) {
   switch (status) {

@@ -161,3 +161,10 @@ def test_deterministic_bwd_without_a_device(lib):
         pytest.skip("a device is present")
     assert lib.fa_bwd_deterministic(P, P, P, P, None, P, P, P, P, P, 1, 2, 256, 64, 0.125, 1, P, 1 << 30,
                                     None) == 5
+
+
+def test_version_encodes_major_minor_patch(lib):
+    v = lib.fa_version()
+    assert v >= 200  # 0.2.0 added fa_bwd_deterministic
+    major, minor, patch = v // 10000, v // 100 % 100, v % 100
+    assert (major, minor, patch) >= (0, 2, 0)
