@@ -25,8 +25,8 @@
  *                                               statistic ("Recomputation")
  *
  * Backward, for an upstream gradient dO (plain chain rule through the three
- * steps above; the pages only say that S_0 and S_1 are recomputed from the
- * stored m and l to get the gradients with respect to Q, K and V):
+ * steps above; the review's "Recomputation" section only states that S_0 and
+ * S_1 are rebuilt from the stored m and l when dQ, dK and dV are computed):
  *
  *   dP_ij = sum_c dO_ic V_jc
  *   D_i   = sum_j P_ij dP_ij
