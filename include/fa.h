@@ -245,11 +245,22 @@ int fa_device_status(void *stream);
 
 /*
  * Like fa_device_status(), and also copies the failure record into info[0..3]:
- * {kernel id (1 fwd, 2 bwd, 4 deterministic dQ), wait tag, block
+ * {kernel id (1 fwd, 2 bwd, 4 deterministic dQ, 5 fa_selftest_timeout), wait tag, block
  * index, launch sequence number}; zeros when there was no failure.  `info` is a
  * host pointer to 4 ints (may be NULL).
  */
 int fa_device_status_info(void *stream, int *info);
+
+/*
+ * Diagnostic of the device-side failure path.  Launches one thread on `stream`
+ * that waits on a pipeline barrier nothing will complete.  Like every wait in
+ * the kernels, that wait is bounded: after its time limit (1 s) the kernel
+ * records FA_ERR_DEVICE_TIMEOUT in the status word (kernel id 5, wait tag 1)
+ * and returns, so the context stays usable.  The next fa_device_status() then
+ * returns FA_ERR_DEVICE_TIMEOUT and clears the word.  Returns FA_OK once the
+ * kernel is launched, or FA_ERR_NO_DEVICE / FA_ERR_UNSUPPORTED / FA_ERR_CUDA.
+ */
+int fa_selftest_timeout(void *stream);
 
 /* Library version, MAJOR*10000 + MINOR*100 + PATCH. */
 int fa_version(void);

@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.fa_device_status.restype = i
         L.fa_device_status_info.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
         L.fa_device_status_info.restype = i
+        L.fa_selftest_timeout.argtypes = [vp]
+        L.fa_selftest_timeout.restype = i
         L.fa_version.argtypes = []
         L.fa_version.restype = i
         _lib = L
@@ -206,6 +208,14 @@ def fa_device_status(stream=None, info: bool = False):
     buf = (ctypes.c_int * 4)()
     rc = lib().fa_device_status_info(_stream_handle(stream), buf)
     return (rc, list(buf)) if info else rc
+
+
+def fa_selftest_timeout(stream=None) -> None:
+    """Launch the failure-path self-test: a wait that gives up after its 1 s limit
+    and records FA_ERR_DEVICE_TIMEOUT, which ``fa_device_status`` then returns."""
+    rc = lib().fa_selftest_timeout(_stream_handle(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_selftest_timeout")
 
 
 class Attention:

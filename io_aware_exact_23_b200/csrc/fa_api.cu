@@ -201,6 +201,28 @@ __global__ void fa_dropout_mask_kernel(uint8_t *mask, long BH, int N, fa::Dropou
   }
 }
 
+// Self-test of the device-side failure path: one thread waits on an mbarrier
+// that nothing arrives on.  The bounded wait gives up after its time limit,
+// records the failure in the status block (kernel kKernelSelftest, wait tag
+// kSelftestTag) and the kernel returns normally, leaving the context usable.
+constexpr int kKernelSelftest = 5;
+constexpr int kSelftestTag = 1;
+
+__global__ void fa_selftest_timeout_kernel(int *status, int seq) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    fa::mbar_init(&bar, 1);
+    fa::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const fa::WaitCtx ctx{status, reinterpret_cast<volatile int *>(&abort_flag), kKernelSelftest, seq};
+    fa::mbar_wait(ctx, &bar, 0, kSelftestTag);
+  }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -399,6 +421,14 @@ int fa_device_status_info(void *stream, int *info) {
 }
 
 int fa_device_status(void *stream) { return fa_device_status_info(stream, nullptr); }
+
+int fa_selftest_timeout(void *stream) {
+  DeviceState *ds = nullptr;
+  const int st = device_state(&ds, nullptr);
+  if (st != FA_OK) return st;
+  fa_selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(ds->status, next_seq());
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
 
 }  // extern "C"
 

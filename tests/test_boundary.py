@@ -168,3 +168,10 @@ def test_version_encodes_major_minor_patch(lib):
     assert v >= 200  # 0.2.0 added fa_bwd_deterministic
     major, minor, patch = v // 10000, v // 100 % 100, v % 100
     assert (major, minor, patch) >= (0, 2, 0)
+
+
+def test_selftest_without_a_device(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    assert lib.fa_selftest_timeout(None) == 5
