@@ -75,3 +75,19 @@ def test_reference_arm_prints_the_contract_line():
         assert key in d, key
     assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["config"]["workload"] == "tiny_b1h2n256d64"
+
+
+def test_variant_arms_are_exclusive_and_need_a_device():
+    """--dropout and --deterministic are separate arms; without a GPU every
+    device arm refuses loudly instead of falling back to the CPU."""
+    import subprocess
+    import sys
+    import torch
+    run = lambda *a: subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *a],  # noqa: E731
+                                    capture_output=True, text=True, timeout=300, cwd=ROOT)
+    both = run("--dropout", "0.1", "--deterministic", "--steps", "1", "--warmup", "1")
+    assert both.returncode != 0 and "separate arms" in both.stderr
+    if not torch.cuda.is_available():
+        for args in (("--deterministic",), ("--dropout", "0.1"), ()):
+            out = run(*args, "--steps", "1", "--warmup", "1", "--no-cpu-baseline")
+            assert out.returncode != 0 and not out.stdout.strip().startswith("{"), args
