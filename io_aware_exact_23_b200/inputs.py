@@ -85,6 +85,32 @@ def make_inputs(w: Workload, device="cpu", with_grad_out: bool = True):
     return out
 
 
+def make_fp8_inputs(w: Workload, device="cpu"):
+    """e4m3 codes of Q, K, V with one fp32 descale factor per head.
+
+    The fp32 draws are those of ``make_inputs`` (same generator, same order,
+    before the bf16 rounding; the stress multiplier applies to Q and K).  Per
+    (b, h) and tensor, descale = max|x| / 448 (448 is e4m3's largest finite
+    value), and the codes are x / descale rounded to nearest even in e4m3
+    (torch's float8_e4m3fn conversion), returned as uint8.  The values the
+    codes stand for are code_value * descale.
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+    shape = (w.B, w.H, w.N, w.d)
+    out = {}
+    for nm in ("q", "k", "v"):
+        x = torch.randn(shape, generator=g, dtype=torch.float32)
+        if nm in ("q", "k") and w.qk_mult != 1.0:
+            x = x * w.qk_mult
+        amax = x.abs().amax(dim=(2, 3)).clamp_min(1e-30)
+        descale = amax / 448.0
+        codes = (x / descale[:, :, None, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+        out[nm] = codes.to(device)
+        out["d" + nm] = descale.to(device)
+    return out
+
+
 def make_shape_inputs(B, H, N, d, seed=0, qk_mult=1.0, device="cpu"):
     """Same recipe for an ad-hoc shape (edge-case tests)."""
     return make_inputs(Workload("adhoc", B, H, N, d, False, qk_mult, seed), device=device)

@@ -5,14 +5,16 @@ baseline leg of ``bench.py`` may import this package; the product path
 (``io_aware_exact_23_b200``) never does, and the two share no code.
 
 ``ref_attn.c`` holds the arithmetic (plain per-row loops in fp64, see its
-header for the passages of the FlashAttention pages it follows);
+header for the passages of the FlashAttention pages it follows); ``fp8.py``
+the e4m3 decoder, the FP8 forward's reference and its P-rounding bound;
 ``ref_numpy.py`` is an independent whole-matrix NumPy restatement used only
 to cross-check the C code on tiny shapes.  This module compiles the C file
 with gcc on first use and marshals arrays through ctypes.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (closed forms, invariants, finite differences, autograd, hand-derived golden
-fixtures).
+fixtures), the dropout functions by ``tests/test_dropout_oracle_pins.py`` and
+``fp8.py`` by ``tests/test_fp8_oracle_pins.py``.
 """
 from __future__ import annotations
 
