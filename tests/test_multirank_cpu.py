@@ -39,7 +39,7 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks():
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of this (multi-threaded) test process
     out = mgr.dict()
     mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
     for r in range(2):
