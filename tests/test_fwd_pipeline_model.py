@@ -177,3 +177,12 @@ def test_model_detects_a_missing_wait():
         except AssertionError:
             failures += 1
     assert failures > 0
+
+
+def test_model_rings_match_the_kernel():
+    """The ring depths this model runs are the kernel's (read from its source)."""
+    import os
+    import re
+    src = open(os.path.join(os.path.dirname(__file__), "..", "io_aware_exact_23_b200", "csrc", "fa_fwd.cuh")).read()
+    m = re.search(r"kStages = \(D == 128\) \? (\d+) : (\d+);", src)
+    assert m and {int(m.group(1)), int(m.group(2))} == {4, 8}
