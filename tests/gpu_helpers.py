@@ -16,6 +16,9 @@ the forward returns.  Every other workload is gated on the strict form.
 """
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -88,6 +91,23 @@ def gate_o(w: Workload, o, o_ref, o_lo=None, label=""):
     return strict, pre, res
 
 
+def record_parity(w: Workload, kind: str, **errs):
+    """Append one JSON line of measured errors to the file named by the
+    FA_PARITY_LOG environment variable (no-op when it is unset).  The strict
+    max|O - O_ref| is recorded beside the pre-rounding and residual errors the
+    stress gate uses, flagged when it exceeds 1e-2."""
+    path = os.environ.get("FA_PARITY_LOG")
+    if not path:
+        return
+    rec = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+           "qk_mult": w.qk_mult, "kind": kind}
+    rec.update({k: (None if v is None else (float(v) if np.isscalar(v) else v)) for k, v in errs.items()})
+    strict = errs.get("strict")
+    rec["strict_over_1e-2"] = bool(strict is not None and strict > TOL_O)
+    with open(path, "a") as f:
+        f.write(json.dumps(rec) + "\n")
+
+
 def to64(x):
     return x.detach().to("cpu", torch.float64).numpy()
 
@@ -122,7 +142,7 @@ def full_check(w: Workload, device="cuda", check_bwd=True, nthreads=0, residual=
     else:
         (o, lse), o_lo = gpu_forward(t, w.scale, w.causal), None
     o_ref, lse_ref = oracle.ref_fwd(t["q"], t["k"], t["v"], w.scale, w.causal, nthreads=nthreads)
-    eo, _, _ = gate_o(w, o, o_ref, o_lo, w.name)
+    eo, epre, eres = gate_o(w, o, o_ref, o_lo, w.name)
     el = max_err(to64(lse), lse_ref)
     assert el <= TOL_LSE, f"{w.name}: max|LSE - LSE_ref| = {el:.3e}"
     out = {"o": eo, "lse": el}
@@ -132,6 +152,8 @@ def full_check(w: Workload, device="cuda", check_bwd=True, nthreads=0, residual=
         check_grads({"dq": to64(dq), "dk": to64(dk), "dv": to64(dv)}, {"dq": rq, "dk": rk, "dv": rv}, w.name)
         for nm, g, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
             out[nm] = max_err(to64(g), r) / max(float(np.abs(r).max()), 1e-30)
+    record_parity(w, "full", strict=eo, pre_rounding=epre, residual=eres, lse=el,
+                  grads_rel={k: out[k] for k in ("dq", "dk", "dv") if k in out})
     return out
 
 

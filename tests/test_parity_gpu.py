@@ -4,8 +4,8 @@ Every input comes from the seeded generator (io_aware_exact_23_b200.inputs);
 every expected value comes from ``oracle``.  Small shapes are compared element
 by element over whole tensors; the full-size workloads are compared at sampled
 (head, row) positions the oracle computes one by one (O, LSE, dQ rows; dK, dV
-rows at the key tiles whose query stats are cheap), plus gradient identities
-that hold at any size:  sum_j dK_j = 0,  sum_j dV_j = sum_i dO_i  and
+rows of one head: the whole head up to N = 4096 -- 1024 in the sweep -- else
+key tiles 0, middle and last), plus gradient identities that hold at any size:  sum_j dK_j = 0,  sum_j dV_j = sum_i dO_i  and
 sum_i Q_i.dQ_i = sum_j K_j.dK_j.
 """
 from __future__ import annotations
@@ -19,7 +19,7 @@ from io_aware_exact_23_b200 import inputs as I
 from io_aware_exact_23_b200.inputs import Workload, make_inputs
 
 from gpu_helpers import (TOL_GRAD_REL, TOL_LSE, TOL_O, full_check, gate_o, gpu_backward, gpu_forward, max_err,
-                         sample_rows, to64)
+                         record_parity, sample_rows, to64)
 
 pytestmark = pytest.mark.gpu
 
@@ -149,7 +149,16 @@ def test_non_default_stream():
 
 
 # ------------------------------------------------------ full-size workloads
-def check_sampled(w: Workload, n_rows=192, dkdv_full_head_max_n=4096, n_tail_keys=128):
+def key_tile_rows(N: int) -> np.ndarray:
+    """Key rows of three 128-row key tiles: tile 0, a middle tile and the last
+    (ragged) tile.  When causal, tile 0 accumulates every query tile and the
+    last tile only the diagonal one; non-causal, each sees every query tile."""
+    nt = (N + 127) // 128
+    tiles = sorted({0, nt // 2, nt - 1})
+    return np.concatenate([np.arange(t * 128, min(N, (t + 1) * 128)) for t in tiles])
+
+
+def check_sampled(w: Workload, n_rows=192, dkdv_full_head_max_n=4096):
     t = make_inputs(w, device="cuda")
     o, lse, o_lo = gpu_forward(t, w.scale, w.causal, residual=True)
     dq, dk, dv = gpu_backward(t, o, lse, w.scale, w.causal, o_lo=o_lo)
@@ -160,30 +169,28 @@ def check_sampled(w: Workload, n_rows=192, dkdv_full_head_max_n=4096, n_tail_key
     o_s = o.reshape(BH, N, d)[sbt, srt]
     olo_s = o_lo.reshape(BH, N, d)[sbt, srt]
     lf = to64(lse).reshape(BH, N)
-    eo, _, _ = gate_o(w, o_s, o_ref, olo_s, w.name + " (sampled)")
+    eo, epre, eres = gate_o(w, o_s, o_ref, olo_s, w.name + " (sampled)")
     el = max_err(lf[sb, sr], l_ref)
     assert el <= TOL_LSE, f"{w.name}: sampled max|LSE-LSE_ref| = {el:.3e}"
     # dQ at the same rows; the gate's scale is the oracle's max over the sampled rows
     dq_ref = oracle.ref_dq_rows(t["q"], t["k"], t["v"], t["do"], w.scale, w.causal, sb, sr)
     dqf = to64(dq).reshape(BH, N, d)
     e = max_err(dqf[sb, sr], dq_ref)
+    rel = {"dq": e / np.abs(dq_ref).max()}
     assert e <= TOL_GRAD_REL * np.abs(dq_ref).max(), f"{w.name}: sampled dQ err {e:.3e}"
-    # dK, dV rows: a whole head when affordable, else the last key tile(s) of a
-    # causal head (their query statistics only need the last rows).
+    # dK, dV rows of one head, element by element: the whole head when it is
+    # affordable, else key tiles 0, middle and last (see key_tile_rows).
     dkf, dvf = to64(dk).reshape(BH, N, d), to64(dv).reshape(BH, N, d)
     head = int(np.random.default_rng(w.N).integers(0, BH))
-    if N <= dkdv_full_head_max_n:
-        keys = np.arange(N)
-    elif w.causal:
-        keys = np.arange(N - n_tail_keys, N)
-    else:
-        keys = None
-    if keys is not None:
-        rk, rv = oracle.ref_dkdv_rows(t["q"], t["k"], t["v"], t["do"], w.scale, w.causal, head, keys)
-        for nm, g, r in (("dK", dkf[head, keys], rk), ("dV", dvf[head, keys], rv)):
-            e = max_err(g, r)
-            assert e <= TOL_GRAD_REL * np.abs(r).max(), f"{w.name}: {nm} err {e:.3e} vs {np.abs(r).max():.3e}"
-    # identities over every head, in fp64 on the GPU outputs
+    keys = np.arange(N) if N <= dkdv_full_head_max_n else key_tile_rows(N)
+    rk, rv = oracle.ref_dkdv_rows(t["q"], t["k"], t["v"], t["do"], w.scale, w.causal, head, keys)
+    for nm, g, r in (("dK", dkf[head, keys], rk), ("dV", dvf[head, keys], rv)):
+        e = max_err(g, r)
+        rel[nm.lower()] = e / np.abs(r).max()
+        assert e <= TOL_GRAD_REL * np.abs(r).max(), f"{w.name}: {nm} err {e:.3e} vs {np.abs(r).max():.3e}"
+    record_parity(w, "sampled", strict=eo, pre_rounding=epre, residual=eres, lse=el, grads_rel=rel,
+                  dkdv_keys=int(len(keys)), head=head)
+    # identities over every head, in fp64 on the GPU outputs (extra checks)
     q64 = t["q"].double()
     k64 = t["k"].double()
     dk64, dv64, dq64 = dk.double(), dv.double(), dq.double()
