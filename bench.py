@@ -19,7 +19,10 @@ data-path collective).  Prints one JSON line on rank 0.
 ``--impl vanilla`` times standard attention (S and P in HBM) on one GPU;
 ``--dropout RATE`` times the step with fused dropout on the probabilities;
 ``--deterministic`` times the step with the deterministic backward;
-``--sweep`` prints one line per workload (forward and backward separately).
+``--sweep`` prints one line per workload (forward and backward separately);
+``--fp8`` times the e4m3 forward (fa_fwd_fp8) on the workload;
+``--max-n`` finds the longest sequence each library runs (fwd + bwd, B=1, H=16,
+d=128, causal): this library and standard attention (``libfa_vanilla.so``).
 """
 from __future__ import annotations
 
@@ -65,6 +68,11 @@ def parse_args():
                     help="time the step with fa_bwd_deterministic (dQ in a fixed summation order)")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="time the fused-dropout step (fa_fwd_dropout + fa_bwd_dropout) at this rate, 1 GPU")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time the e4m3 forward (fa_fwd_fp8) on the workload (d = 128), 1 GPU")
+    ap.add_argument("--max-n", action="store_true",
+                    help="longest sequence (B=1, H=16, d=128, causal, fwd + bwd) that runs, for this library and "
+                         "for standard attention; 1 GPU")
     return ap.parse_args()
 
 
@@ -449,13 +457,195 @@ def run_sweep(args):
     return 0
 
 
+def run_fp8(args, w):
+    """--fp8 (1 GPU): the e4m3 forward, fa_fwd_fp8, timed with CUDA events.  Its
+    peak is the measured bf16 dense peak x 2 (the nominal e4m3 : bf16 ratio of
+    the tensor cores)."""
+    import torch
+    from io_aware_exact_23_b200 import binding as fa
+    from io_aware_exact_23_b200.inputs import make_fp8_inputs
+    if w.d != 128:
+        raise SystemExit("bench.py: the e4m3 forward takes d = 128")
+    dev = torch.device("cuda:0")
+    t = make_fp8_inputs(w, device=dev)
+    B, H, N, d = w.B, w.H, w.N, w.d
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+
+    def step():
+        fa.fa_fwd_fp8(t["q"], t["k"], t["v"], t["dq"], t["dk"], t["dv"], o, lse, w.scale, w.causal)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    K = args.steps
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    start, end = mk(), mk()
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(K):
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    if fa.fa_device_status() != 0:
+        raise SystemExit("bench.py: device status error")
+    ms = start.elapsed_time(end) / K
+    peaks, peak_kind = load_peaks()
+    peak = 2.0 * float(peaks["bf16_tflops"])
+    tf = w.fwd_flops() / (ms / 1e3) / 1e12
+    in_bytes = 3 * B * H * N * d
+    line = {"metric": METRIC, "value": tf, "unit": UNIT, "impl": "ours", "n_gpus": 1, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3 in, fp32 accumulate, bf16 out", "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
+                       "step": "fa_fwd_fp8 (forward only)", "l2": f"inputs {in_bytes / 1e6:.0f} MB"},
+            "roofline": {"bound": "tensor", "kernel": "fa_fwd_kernel<128, causal, 0, fp8>", "achieved": tf,
+                         "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                         "peak_kind": f"e4m3 dense = 2 x bf16 dense burst ({peak_kind}), the nominal ratio"},
+            "gpu_launches": K}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_max_n(args):
+    """--max-n (1 GPU): the longest sequence that runs one fwd + bwd step at B=1,
+    H=16, d=128, causal -- for this library (fa_fwd with the residual + fa_bwd)
+    and for standard attention (libfa_vanilla.so, S and P in HBM).  N doubles
+    from 8192 until the step cannot run (the allocation fails, or the library
+    refuses the shape); the largest N whose tensors allocate is then bisected
+    to a multiple of 1024, and the step is run there.  Inputs are N(0,1) bf16
+    drawn on the device from a seeded generator (a capacity probe: only the
+    sizes matter)."""
+    import torch
+    from io_aware_exact_23_b200 import binding as fa
+    from io_aware_exact_23_b200 import vanilla
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    torch.zeros(1, device=dev)
+    total = torch.cuda.get_device_properties(dev).total_memory
+    B, H, d, scale = 1, 16, 128, 1.0 / 128 ** 0.5
+
+    def alloc(impl, N):
+        """The step's tensors, or the reason they cannot exist."""
+        if impl == "ours":
+            wsb = fa.fa_bwd_workspace_bytes(B, H, N, d)
+            if wsb == 0:
+                return None, "refused by the library: B*H*N*d >= 2^31 elements per tensor"
+        else:
+            wsb = vanilla.workspace_bytes(B, H, N, d)
+            if wsb == 0:
+                return None, "refused by the library"
+        try:
+            g = torch.Generator(device=dev)
+            g.manual_seed(N)
+            T = {nm: torch.randn((B, H, N, d), generator=g, device=dev, dtype=torch.bfloat16)
+                 for nm in ("q", "k", "v", "do")}
+            for nm in ("o", "dq", "dk", "dv") + (("o_lo",) if impl == "ours" else ()):
+                T[nm] = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+            T["lse"] = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+            T["ws"] = torch.empty(wsb, dtype=torch.uint8, device=dev)
+            return T, None
+        except torch.cuda.OutOfMemoryError:
+            return None, "out of memory (torch allocation)"
+
+    def run(impl, N, T):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        try:
+            e0.record()
+            if impl == "ours":
+                fa.fa_fwd(T["q"], T["k"], T["v"], T["o"], T["lse"], scale, True, o_lo=T["o_lo"])
+                fa.fa_bwd(T["q"], T["k"], T["v"], T["o"], T["do"], T["lse"], T["dq"], T["dk"], T["dv"], scale, True,
+                          T["ws"], o_lo=T["o_lo"])
+            else:
+                vanilla.fwd(T["q"], T["k"], T["v"], T["o"], T["lse"], scale, True, T["ws"])
+                vanilla.bwd(T["q"], T["k"], T["v"], T["o"], T["do"], T["lse"], T["dq"], T["dk"], T["dv"], scale, True,
+                            T["ws"])
+            e1.record()
+            torch.cuda.synchronize()
+        except Exception as ex:  # a library status code (e.g. cuBLAS could not allocate)
+            torch.cuda.synchronize()
+            return None, f"call failed: {ex}"
+        if impl == "ours" and fa.fa_device_status() != 0:
+            return None, "device status error"
+        finite = bool(torch.isfinite(T["dq"].float()).all() and torch.isfinite(T["o"].float()).all())
+        return {"ms": e0.elapsed_time(e1), "finite": finite}, None
+
+    def free():
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+    for impl in ("ours", "vanilla"):
+        tried = []
+        N, ok_n, fail_n, fail_why = 8192, None, None, None
+        while True:
+            T, why = alloc(impl, N)
+            r = None
+            if T is not None:
+                torch.cuda.reset_peak_memory_stats(dev)
+                r, why = run(impl, N, T)
+                peak = torch.cuda.max_memory_allocated(dev)
+            del T
+            free()
+            tried.append({"N": N, "ok": r is not None, "ms": r and r["ms"], "why": why})
+            if r is None:
+                fail_n, fail_why = N, why
+                break
+            ok_n = N
+            N *= 2
+        # bisect the largest N whose tensors exist (allocation or the library's shape check)
+        lo, hi = ok_n or 0, fail_n
+        while hi - lo > 1024:
+            mid = (lo + hi) // 2 // 1024 * 1024
+            if mid <= lo:
+                break
+            T, why = alloc(impl, mid)
+            good = T is not None
+            del T
+            free()
+            lo, hi = (mid, hi) if good else (lo, mid)
+        if impl == "ours" and fa.fa_bwd_workspace_bytes(B, H, hi - 1, d) != 0:
+            lo = hi - 1  # the library's limit is exact: the last N it accepts
+        # run the step at the largest N that allocates (stepping down if the call itself fails)
+        best, best_rec = None, None
+        n_try = lo
+        while n_try >= (ok_n or 0) and n_try > 0:
+            T, why = alloc(impl, n_try)
+            if T is not None:
+                torch.cuda.reset_peak_memory_stats(dev)
+                r, why = run(impl, n_try, T)
+                peak = torch.cuda.max_memory_allocated(dev)
+            else:
+                r = None
+            del T
+            free()
+            tried.append({"N": n_try, "ok": r is not None, "ms": r and r["ms"], "why": why})
+            if r is not None:
+                best, best_rec = n_try, {**r, "peak_hbm_bytes": peak}
+                break
+            n_try -= 1024
+        flops = 14.0 * B * H * best * best * d / 2 if best else 0.0  # fwd + bwd, causal
+        line = {"probe": "max_n", "impl": impl, "B": B, "H": H, "d": d, "causal": True,
+                "step": ("fa_fwd (with the residual) + fa_bwd" if impl == "ours" else
+                         "standard attention fwd + bwd (S fp32, P bf16 in HBM)"),
+                "max_n_run": best, "step_ms": best_rec and best_rec["ms"],
+                "step_tflops": (flops / (best_rec["ms"] / 1e3) / 1e12) if best_rec else None,
+                "peak_hbm_bytes": best_rec and best_rec["peak_hbm_bytes"], "device_memory_bytes": total,
+                "outputs_finite": best_rec and best_rec["finite"],
+                "first_failure": {"N": fail_n, "why": fail_why}, "tried": tried}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     world, rank, local = dist_setup()
     from io_aware_exact_23_b200.inputs import CONFIGS
     if args.sweep:
         return run_sweep(args)
+    if args.max_n:
+        return run_max_n(args)
     w = CONFIGS[args.workload]
+    if args.fp8:
+        return run_fp8(args, w)
     if args.impl == "reference":
         return run_reference(args, w, world, rank)
     if args.impl == "vanilla":
@@ -604,6 +794,10 @@ def main():
                          "frac_of_sustained": dom_tf / peak_sus,
                          "traffic": stored_traffic(dominant, w.name)},
             "peak_hbm_bytes": peak_mem,
+            # libfa.so's device image, resident on every GPU that loads it, outside
+            # torch's allocator: the no-alloc backward's static scratch array plus
+            # its status word (and the 32-byte allocated status block).
+            "library_resident_bytes": fa.NOALLOC_SCRATCH_BYTES + 32 + 32,
             "score_matrix_bytes_bf16": score_matrix_bytes(B, H, N, 2),
             "clocks": clocks,
             "gpu_launches": 4 * K,

@@ -111,6 +111,28 @@ int fa_fwd_residual(const void *q, const void *k, const void *v, void *o,
                     float scale, int causal, void *stream);
 
 /*
+ * FP8 forward pass (the FlashAttention topic page names FP8 as a
+ * FlashAttention-3 feature, "FlashAttention-3 (2024)", without a scheme).
+ * Inputs are e4m3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits;
+ * the "fn" variant without infinities) with one fp32 descale factor per head:
+ *   q8, k8, v8           [B, H, N, d] uint8 e4m3 codes (device, 16-byte aligned)
+ *   descale_q/_k/_v      [B, H] fp32 (device, 4-byte aligned); the inputs are the
+ *                        reals code_value * descale
+ *   o                    [B, H, N, d] bf16 output, lse [B, H, N] fp32 (natural log)
+ * It computes O = softmax(scale * Q K^T [+ causal mask]) V of those reals, as
+ * fa_fwd does, with two differences of precision: S = Q K^T accumulates the
+ * exact e4m3 products in fp32, and the probabilities P are rounded to e4m3
+ * (relative error <= 2^-4, absolute <= 2^-10 below 2^-6) before the PV
+ * product; O is divided by the fp32 row sum of the unrounded P, and lse is
+ * that of the unrounded P.  Supported: d = 128 only (FA_ERR_UNSUPPORTED
+ * otherwise); other arguments, errors and ownership as fa_fwd.
+ */
+int fa_fwd_fp8(const void *q8, const void *k8, const void *v8,
+               const float *descale_q, const float *descale_k,
+               const float *descale_v, void *o, float *lse, int B, int H,
+               int N, int d, float scale, int causal, void *stream);
+
+/*
  * Forward pass with dropout on the attention probabilities (the fused dropout
  * the FlashAttention pages count among the method's largest speed-ups): the
  * same arguments as fa_fwd_residual (o_lo may be NULL), plus
@@ -182,9 +204,10 @@ int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o,
  * recomputes S_ij = Q_i K_j^T, P_ij (from LSE, as in the review's
  * "Recomputation" section), dP_ij = dO_i V_j^T and dS_ij (the chain rule
  * through softmax) and sums dQ_i over the key tiles in ascending j in tensor
- * memory.  dK and dV come from the fused kernel, bit for bit as in fa_bwd.
- * Costs about 1.6x fa_bwd's tensor-core work (the fused kernel's own dQ product
- * is still computed and discarded).
+ * memory.  dK and dV come from the fused kernel run without its dQ product, bit
+ * for bit as in fa_bwd (the same products in the same order).  Costs 7 tile
+ * products per (query tile, key tile) pair against fa_bwd's 5: 1.4x the
+ * tensor-core work.
  *
  * Arguments, layout, ownership and errors: as fa_bwd_ex with events = NULL
  * (o_lo may be NULL); the workspace size is fa_bwd_workspace_bytes(B, H, N, d).
@@ -223,14 +246,35 @@ int fa_bwd_deterministic(const void *q, const void *k, const void *v,
  * whose kernels overlap on the GPU -- on different streams, or from different
  * host threads -- race on the array and must be serialised by the caller.
  * A device-side wait timeout in these kernels is recorded in a status word that
- * also lives in the static image; fa_device_status() does not see it (it owns
- * a separately allocated word), and dq/dk/dv are then undefined.
+ * also lives in the static image (dq/dk/dv are then undefined).
+ * fa_device_status() does not see that word (it owns a separately allocated
+ * one): read it with fa_noalloc_device_status() after the call.
  */
 #define FA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
                    const void *dO, const float *lse, void *dq, void *dk,
                    void *dv, int B, int H, int N, int d, float scale,
                    int causal, void *stream);
+
+/*
+ * The failure record of fa_bwd_noalloc: synchronises `stream`, then returns and
+ * clears the status word in the static image that fa_bwd_noalloc's kernels
+ * write -- FA_OK, or FA_ERR_DEVICE_TIMEOUT if one of them gave up on a wait
+ * since the last read (its dq/dk/dv are then undefined) -- and copies the
+ * record into info[0..3] as fa_device_status_info() does (info may be NULL).
+ * Allocates nothing; the first no-alloc call on a device does the same
+ * one-time set-up as fa_bwd_noalloc.  FA_ERR_CUDA if a CUDA call fails.
+ */
+int fa_noalloc_device_status(void *stream, int *info);
+
+/*
+ * fa_selftest_timeout() aimed at fa_bwd_noalloc's status word: one thread
+ * waits on a barrier nothing completes, gives up after 1 s and records
+ * FA_ERR_DEVICE_TIMEOUT (kernel id 5, wait tag 1) there, so that
+ * fa_noalloc_device_status() can be checked without a fault.  Allocates
+ * nothing.
+ */
+int fa_noalloc_selftest_timeout(void *stream);
 
 /* Static, human-readable name of a status code (never NULL). */
 const char *fa_status_string(int status);

@@ -52,6 +52,8 @@ def lib() -> ctypes.CDLL:
                                 ctypes.POINTER(vp)]
         L.fa_bwd_ex.restype = i
         u64, u32 = ctypes.c_ulonglong, ctypes.c_uint
+        L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+        L.fa_fwd_fp8.restype = i
         L.fa_fwd_dropout.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, f, u64, u32, vp]
         L.fa_fwd_dropout.restype = i
         L.fa_bwd_dropout.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, f, u64, u32, vp, sz,
@@ -73,6 +75,10 @@ def lib() -> ctypes.CDLL:
         L.fa_device_status_info.restype = i
         L.fa_selftest_timeout.argtypes = [vp]
         L.fa_selftest_timeout.restype = i
+        L.fa_noalloc_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+        L.fa_noalloc_device_status.restype = i
+        L.fa_noalloc_selftest_timeout.argtypes = [vp]
+        L.fa_noalloc_selftest_timeout.restype = i
         L.fa_version.argtypes = []
         L.fa_version.restype = i
         _lib = L
@@ -120,6 +126,25 @@ def fa_fwd(q, k, v, o, lse, scale: float, causal: bool, stream=None, o_lo=None) 
                                    _stream_handle(stream))
     if rc != FA_OK:
         raise FaError(rc, "fa_fwd")
+
+
+def fa_fwd_fp8(q8, k8, v8, descale_q, descale_k, descale_v, o, lse, scale: float, causal: bool,
+               stream=None) -> None:
+    """FP8 forward: ``q8``, ``k8``, ``v8`` are uint8 e4m3 codes [B,H,N,d] (d = 128),
+    ``descale_*`` fp32 [B,H] per-head factors (inputs = code * descale); O into the
+    bf16 ``o`` [B,H,N,d] and LSE into the fp32 ``lse`` [B,H,N]."""
+    B, H, N, d = q8.shape
+    for nm, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        _check(t, nm, torch.uint8, (B, H, N, d))
+    for nm, t in (("descale_q", descale_q), ("descale_k", descale_k), ("descale_v", descale_v)):
+        _check(t, nm, torch.float32, (B, H))
+    _check(o, "o", torch.bfloat16, (B, H, N, d))
+    _check(lse, "lse", torch.float32, (B, H, N))
+    rc = lib().fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), descale_q.data_ptr(), descale_k.data_ptr(),
+                          descale_v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, N, d, float(scale),
+                          int(bool(causal)), _stream_handle(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_fp8")
 
 
 def fa_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
@@ -201,6 +226,20 @@ def fa_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, scale: float, causal: bool, 
                               float(scale), int(bool(causal)), _stream_handle(stream))
     if rc != FA_OK:
         raise FaError(rc, "fa_bwd_noalloc")
+
+
+def fa_noalloc_device_status(stream=None, info: bool = False):
+    """Synchronise the stream and return (and clear) fa_bwd_noalloc's own status code."""
+    buf = (ctypes.c_int * 4)()
+    rc = lib().fa_noalloc_device_status(_stream_handle(stream), buf)
+    return (rc, list(buf)) if info else rc
+
+
+def fa_noalloc_selftest_timeout(stream=None) -> None:
+    """The failure-path self-test aimed at fa_bwd_noalloc's status word."""
+    rc = lib().fa_noalloc_selftest_timeout(_stream_handle(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_noalloc_selftest_timeout")
 
 
 def fa_device_status(stream=None, info: bool = False):

@@ -1,6 +1,6 @@
 """Build libfa.so (the C-ABI attention library) in-tree with nvcc for sm_100a.
 
-Usage: ``python -m io_aware_exact_23_b200.build [--force] [--debug-bounds]``.
+Usage: ``python -m io_aware_exact_23_b200.build [--force] [-v]``.
 The library is written next to this file so that it travels with the source
 tree; nothing is installed into site-packages.
 """

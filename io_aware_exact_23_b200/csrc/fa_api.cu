@@ -77,6 +77,11 @@ int encode_bf16(CUtensorMap *m, const void *ptr, int D, int N, int BH) {
   return encode_3d(m, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, BH, 64);
 }
 
+// e4m3 codes as bytes: 128-element (128-byte) box rows.
+int encode_u8(CUtensorMap *m, const void *ptr, int D, int N, int BH) {
+  return encode_3d(m, ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D, N, BH, 128);
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Shape checks shared by both passes (no CUDA calls).
@@ -90,10 +95,10 @@ int check_shape(int B, int H, int N, int d, float scale, int causal) {
   return FA_OK;
 }
 
-template <int D, bool CAUSAL, bool DROPOUT>
+template <int D, bool CAUSAL, bool DROPOUT, bool FP8 = false>
 cudaError_t fwd_set_attribute() {
-  return cudaFuncSetAttribute(fa::fa_fwd_kernel<D, CAUSAL, DROPOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              fa::FwdCfg<D>::kSmemBytes);
+  return cudaFuncSetAttribute(fa::fa_fwd_kernel<D, CAUSAL, DROPOUT, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              fa::FwdCfg<D, FP8>::kSmemBytes);
 }
 
 // Dropout rate -> the generator's threshold and the kept entries' scale.
@@ -154,6 +159,8 @@ int device_state(DeviceState **out, int *dev_out) {
     e = (e == cudaSuccess) ? fwd_set_attribute<64, true, true>() : e;
     e = (e == cudaSuccess) ? fwd_set_attribute<128, false, true>() : e;
     e = (e == cudaSuccess) ? fwd_set_attribute<128, true, true>() : e;
+    e = (e == cudaSuccess) ? fwd_set_attribute<128, false, false, true>() : e;
+    e = (e == cudaSuccess) ? fwd_set_attribute<128, true, false, true>() : e;
     e = (e == cudaSuccess) ? fa::bwd_set_attributes() : e;
     e = (e == cudaSuccess) ? fa::dq_set_attributes() : e;
     if (e != cudaSuccess) {
@@ -167,12 +174,12 @@ int device_state(DeviceState **out, int *dev_out) {
   return FA_OK;
 }
 
-template <int D, bool CAUSAL, bool DROPOUT>
+template <int D, bool CAUSAL, bool DROPOUT, bool FP8 = false>
 cudaError_t launch_fwd(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v, const CUtensorMap &o,
                        const CUtensorMap &olo, const fa::FwdParams &p, cudaStream_t stream) {
   const dim3 grid(static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.n_qpairs));
-  fa::fa_fwd_kernel<D, CAUSAL, DROPOUT>
-      <<<grid, fa::FwdCfg<D>::kThreads, fa::FwdCfg<D>::kSmemBytes, stream>>>(q, k, v, o, olo, p);
+  fa::fa_fwd_kernel<D, CAUSAL, DROPOUT, FP8>
+      <<<grid, fa::FwdCfg<D, FP8>::kThreads, fa::FwdCfg<D, FP8>::kSmemBytes, stream>>>(q, k, v, o, olo, p);
   return cudaGetLastError();
 }
 
@@ -255,9 +262,49 @@ static int fwd_common(const void *q, const void *k, const void *v, void *o, void
   p.n_qpairs = (N + 255) / 256;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.drop = drop ? *drop : fa::DropoutParams{0u, 0u, 0u, 0u, 1.f};
+  p.descale_q = p.descale_k = p.descale_v = nullptr;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const cudaError_t e = drop ? launch_fwd_any<true>(d, causal, tq, tk, tv, to, tolo, p, s)
                              : launch_fwd_any<false>(d, causal, tq, tk, tv, to, tolo, p, s);
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// e4m3 forward: Q, K, V as byte codes with per-head descale factors; O bf16.
+static int fwd_fp8_common(const void *q8, const void *k8, const void *v8, const float *dq, const float *dk,
+                          const float *dv, void *o, float *lse, int B, int H, int N, int d, float scale, int causal,
+                          void *stream) {
+  if (!q8 || !k8 || !v8 || !dq || !dk || !dv || !o || !lse) return FA_ERR_INVALID_ARG;
+  int st = check_shape(B, H, N, d, scale, causal);
+  if (st != FA_OK) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) || !aligned16(lse) ||
+      (reinterpret_cast<uintptr_t>(dq) & 3u) || (reinterpret_cast<uintptr_t>(dk) & 3u) ||
+      (reinterpret_cast<uintptr_t>(dv) & 3u))
+    return FA_ERR_MISALIGNED;
+  DeviceState *ds = nullptr;
+  st = device_state(&ds, nullptr);
+  if (st != FA_OK) return st;
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv, to;
+  if (encode_u8(&tq, q8, d, N, BH) || encode_u8(&tk, k8, d, N, BH) || encode_u8(&tv, v8, d, N, BH) ||
+      encode_bf16(&to, o, d, N, BH))
+    return FA_ERR_CUDA;
+  fa::FwdParams p;
+  p.lse = lse;
+  p.o_lo = nullptr;
+  p.status = ds->status;
+  p.seq = next_seq();
+  p.N = N;
+  p.BH = BH;
+  p.n_qpairs = (N + 255) / 256;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.drop = fa::DropoutParams{0u, 0u, 0u, 0u, 1.f};
+  p.descale_q = dq;
+  p.descale_k = dk;
+  p.descale_v = dv;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = causal ? launch_fwd<128, true, false, true>(tq, tk, tv, to, to, p, s)
+                               : launch_fwd<128, false, false, true>(tq, tk, tv, to, to, p, s);
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -305,7 +352,7 @@ static int bwd_common(const void *q, const void *k, const void *v, const void *o
 
 extern "C" {
 
-int fa_version(void) { return 200; }  // 0.2.0: fa_bwd_deterministic
+int fa_version(void) { return 300; }  // 0.3.0: fa_fwd_fp8, the no-alloc status reader
 
 const char *fa_status_string(int status) {
   switch (status) {
@@ -330,6 +377,12 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
 int fa_fwd_residual(const void *q, const void *k, const void *v, void *o, void *o_lo, float *lse, int B, int H,
                     int N, int d, float scale, int causal, void *stream) {
   return fwd_common(q, k, v, o, o_lo, lse, B, H, N, d, scale, causal, nullptr, stream);
+}
+
+int fa_fwd_fp8(const void *q8, const void *k8, const void *v8, const float *descale_q, const float *descale_k,
+               const float *descale_v, void *o, float *lse, int B, int H, int N, int d, float scale, int causal,
+               void *stream) {
+  return fwd_fp8_common(q8, k8, v8, descale_q, descale_k, descale_v, o, lse, B, H, N, d, scale, causal, stream);
 }
 
 int fa_fwd_dropout(const void *q, const void *k, const void *v, void *o, void *o_lo, float *lse, int B, int H, int N,
@@ -523,4 +576,45 @@ extern "C" int fa_bwd_noalloc(const void *q, const void *k, const void *v, const
     return FA_ERR_CUDA;
   cudaError_t e = fa::bwd_launch(L, maps, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// The no-alloc path's failure record: its kernels write device-side wait
+// timeouts into fa_noalloc_status (in the static image), which the separately
+// allocated word read by fa_device_status() never sees.  These two calls read
+// and clear that word, and exercise it with the bounded-wait self-test.  Like
+// fa_bwd_noalloc, neither allocates device memory.
+extern "C" int fa_noalloc_device_status(void *stream, int *info) {
+  if (info) std::memset(info, 0, 4 * sizeof(int));
+  NoAllocState *ns = nullptr;
+  int st = noalloc_state(&ns);
+  if (st != FA_OK) return st;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int h[kStatusInts];
+  if (cudaStreamSynchronize(s) != cudaSuccess ||
+      cudaMemcpyAsync(h, ns->status, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  if (h[0] == 0) return FA_OK;
+  if (info) {
+    info[0] = h[1];
+    info[1] = h[2];
+    info[2] = h[3];
+    info[3] = h[4];
+  }
+  if (cudaMemsetAsync(ns->status, 0, kStatusInts * sizeof(int), s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  return h[0] == fa::kStatusInternal ? FA_ERR_DEVICE_INTERNAL : FA_ERR_DEVICE_TIMEOUT;
+}
+
+extern "C" int fa_noalloc_selftest_timeout(void *stream) {
+  NoAllocState *ns = nullptr;
+  const int st = noalloc_state(&ns);
+  if (st != FA_OK) return st;
+  fa_selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(ns->status, next_seq());
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

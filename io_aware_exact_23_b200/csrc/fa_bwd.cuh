@@ -167,6 +167,7 @@ __global__ void __launch_bounds__(256, 4) fa_bwd_pre_kernel(const uint16_t *__re
       }
     }
   }
+  if (ws_dq == nullptr) return;  // no dQ accumulator to zero (the deterministic mode)
   const long n4 = static_cast<long>(BH) * N * D / 4;
   const long tid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long nthreads = static_cast<long>(gridDim.x) * blockDim.x;
@@ -198,7 +199,12 @@ __global__ void __launch_bounds__(256) fa_dq_convert_kernel(const float *__restr
 }
 
 // ------------------------------------------------------------ main kernel
-template <int D, bool CAUSAL, bool DROPOUT = false>
+// NO_DQ: the instantiation of the deterministic mode, whose dQ comes from
+// fa_dq_kernel.  It skips the dQ product and its drain; dK(i) then closes each
+// query tile (its commit takes the place of dQ(i)'s), the issue order is
+// S^T(0) dP^T(0) | dV(i) S^T(i+1) dK(i) dP^T(i+1) | ... at both head dims, and
+// the drain warps' leader only hands each Q_i / dO_i stage back to the producer.
+template <int D, bool CAUSAL, bool DROPOUT = false, bool NO_DQ = false>
 __global__ void __launch_bounds__(448, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -380,7 +386,34 @@ __global__ void __launch_bounds__(448, 1)
       // the compute warps have turned into dS(i): neither waits for an MMA to
       // complete, since one thread issues them all and the pipe runs them in order.
       bool ok = mbar_wait(ctx, bar_kv, 0, kBTagKV);
-      if (D == 128) {
+      if (NO_DQ) {
+        // S^T(0) dP^T(0) | dV(i) S^T(i+1) dK(i) dP^T(i+1) | ...: no dQ in TMEM, so
+        // nothing waits for a drain; dK(i)'s commit closes the tile.
+        ok = ok && wait_stage(0);
+        if (ok) {
+          tc_fence_after();
+          issue_sT(0);
+          issue_dPT(0);
+        }
+        for (int it = 0; it < n_it && ok; ++it) {
+          ok = mbar_wait(ctx, bar_p_full, it & 1, kBTagPFull);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dV(it);
+          if (it + 1 < n_it) {
+            ok = wait_stage(it + 1);
+            if (!ok) break;
+            tc_fence_after();
+            issue_sT(it + 1);
+          }
+          ok = mbar_wait(ctx, bar_ds_full, it & 1, kBTagDsFull);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dK(it);
+          mma_commit(bar_dkq_done);
+          if (it + 1 < n_it) issue_dPT(it + 1);
+        }
+      } else if (D == 128) {
         // Order S^T(i) dP^T(i) dV(i) dK(i) dQ(i).  dQ(i) accumulates in dP^T's
         // columns, so dP^T(i+1) also waits for the drain to have read dQ(i).
         for (int it = 0; it < n_it && ok; ++it) {
@@ -590,6 +623,20 @@ __global__ void __launch_bounds__(448, 1)
       }
     }
     __syncwarp();
+  } else if (NO_DQ) {
+    // --------------------------------------- stage release (no dQ to drain)
+    // The stage of query tile it is free once every MMA issued up to dK(it) --
+    // among them the four that read Q_i and dO_i -- has completed.
+    if (warp == 8 && lane == 0) {
+      bool ok = !*abort_flag;
+      for (int it = 0; it < n_it && ok; ++it) {
+        ok = mbar_wait(ctx, bar_dkq_done, it & 1, kBTagDkqDone);
+        if (!ok) break;
+        mbar_arrive(&bar_qdo_empty[it & 1]);
+        if (it == n_it - 1) mbar_arrive(bar_drained);
+      }
+    }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ dQ drain
     // Staging: the fp32 dQ tile is 128 rows x D columns = 4 * D * 128 bytes, split
@@ -684,27 +731,30 @@ struct BwdLaunch {
   const DropoutParams *drop = nullptr;  // dropout on the probabilities, or none
 };
 
-template <int D, bool CAUSAL, bool DROPOUT>
+template <int D, bool CAUSAL, bool DROPOUT, bool NO_DQ = false>
 inline cudaError_t bwd_set_attribute() {
-  return cudaFuncSetAttribute(fa_bwd_kernel<D, CAUSAL, DROPOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(fa_bwd_kernel<D, CAUSAL, DROPOUT, NO_DQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               BwdCfg<D>::kSmemBytes);
 }
 
 inline cudaError_t bwd_set_attributes() {
-  const cudaError_t es[8] = {bwd_set_attribute<64, false, false>(), bwd_set_attribute<64, true, false>(),
-                             bwd_set_attribute<128, false, false>(), bwd_set_attribute<128, true, false>(),
-                             bwd_set_attribute<64, false, true>(), bwd_set_attribute<64, true, true>(),
-                             bwd_set_attribute<128, false, true>(), bwd_set_attribute<128, true, true>()};
+  const cudaError_t es[12] = {bwd_set_attribute<64, false, false>(), bwd_set_attribute<64, true, false>(),
+                              bwd_set_attribute<128, false, false>(), bwd_set_attribute<128, true, false>(),
+                              bwd_set_attribute<64, false, true>(), bwd_set_attribute<64, true, true>(),
+                              bwd_set_attribute<128, false, true>(), bwd_set_attribute<128, true, true>(),
+                              bwd_set_attribute<64, false, false, true>(), bwd_set_attribute<64, true, false, true>(),
+                              bwd_set_attribute<128, false, false, true>(),
+                              bwd_set_attribute<128, true, false, true>()};
   for (cudaError_t e : es)
     if (e != cudaSuccess) return e;
   return cudaSuccess;
 }
 
-template <int D, bool CAUSAL, bool DROPOUT>
+template <int D, bool CAUSAL, bool DROPOUT, bool NO_DQ = false>
 inline void bwd_main_launch(const CUtensorMap *m, const BwdParams &p, int nkv, cudaStream_t s) {
   const dim3 grid(static_cast<unsigned>(p.BH) * static_cast<unsigned>(nkv));
-  fa_bwd_kernel<D, CAUSAL, DROPOUT><<<grid, BwdCfg<D>::kThreads, BwdCfg<D>::kSmemBytes, s>>>(m[0], m[1], m[2], m[3],
-                                                                                               m[4], m[5], m[6], p);
+  fa_bwd_kernel<D, CAUSAL, DROPOUT, NO_DQ><<<grid, BwdCfg<D>::kThreads, BwdCfg<D>::kSmemBytes, s>>>(
+      m[0], m[1], m[2], m[3], m[4], m[5], m[6], p);
 }
 
 // maps: Q, K, V, dO, dK, dV (bf16, 3-D, 64-feature boxes), dQ accumulator

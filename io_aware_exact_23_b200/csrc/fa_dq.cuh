@@ -389,15 +389,16 @@ inline cudaError_t bwd_launch_deterministic(const BwdLaunch &L, const CUtensorMa
   float *ws_lse2 = ws_dq + static_cast<size_t>(L.BH) * L.N * L.d;
   float *ws_D = ws_lse2 + static_cast<size_t>(L.BH) * Npad;
   const int pre_grid = L.num_sms * 8;
+  // No dQ accumulator here (dQ comes from fa_dq_kernel): nullptr skips its zeroing.
   if (L.d == 64)
     fa_bwd_pre_kernel<64><<<pre_grid, 256, 0, s>>>(static_cast<const uint16_t *>(L.o),
                                                    static_cast<const uint16_t *>(L.o_lo),
-                                                   static_cast<const uint16_t *>(L.dO), L.lse, ws_D, ws_lse2, ws_dq,
+                                                   static_cast<const uint16_t *>(L.dO), L.lse, ws_D, ws_lse2, nullptr,
                                                    L.N, Npad, L.BH);
   else
     fa_bwd_pre_kernel<128><<<pre_grid, 256, 0, s>>>(static_cast<const uint16_t *>(L.o),
                                                     static_cast<const uint16_t *>(L.o_lo),
-                                                    static_cast<const uint16_t *>(L.dO), L.lse, ws_D, ws_lse2, ws_dq,
+                                                    static_cast<const uint16_t *>(L.dO), L.lse, ws_D, ws_lse2, nullptr,
                                                     L.N, Npad, L.BH);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -414,11 +415,13 @@ inline cudaError_t bwd_launch_deterministic(const BwdLaunch &L, const CUtensorMa
   p.scale_log2 = L.scale * 1.4426950408889634f;
   p.scale = L.scale;
   const int nkv = Npad / 128;
+  // dK, dV from the fused kernel without its dQ product (NO_DQ).
   if (L.d == 64)
-    L.causal ? bwd_main_launch<64, true, false>(maps, p, nkv, s) : bwd_main_launch<64, false, false>(maps, p, nkv, s);
+    L.causal ? bwd_main_launch<64, true, false, true>(maps, p, nkv, s)
+             : bwd_main_launch<64, false, false, true>(maps, p, nkv, s);
   else
-    L.causal ? bwd_main_launch<128, true, false>(maps, p, nkv, s)
-             : bwd_main_launch<128, false, false>(maps, p, nkv, s);
+    L.causal ? bwd_main_launch<128, true, false, true>(maps, p, nkv, s)
+             : bwd_main_launch<128, false, false, true>(maps, p, nkv, s);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   DqParams q;

@@ -58,13 +58,24 @@ struct FwdParams {
   int n_qpairs;      // ceil(N / 256)
   float scale_log2;  // scale * log2(e)
   DropoutParams drop;  // read only by the DROPOUT instantiations
+  // FP8 instantiations only: per-head descale factors [BH] of the e4m3 Q, K, V
+  // (the inputs are code * descale).
+  const float *descale_q, *descale_k, *descale_v;
 };
 
-template <int D>
+// FP8: Q, K, V as e4m3 (one byte per element); the output O stays bf16.
+template <int D, bool FP8 = false>
 struct FwdCfg {
-  static constexpr int kTileBytes = 128 * D * 2;      // one 128 x D bf16 tile
-  static constexpr int kStages = (D == 128) ? 4 : 8;  // K/V ring depth (>= 4: the epilogue stages in it)
-  static constexpr int kBoxes = D / 64;               // 64-column TMA boxes per tile
+  static_assert(!FP8 || D == 128, "the e4m3 forward takes d = 128 (one 128-byte swizzle row per tile row)");
+  static constexpr int kElemBytes = FP8 ? 1 : 2;
+  static constexpr int kTileBytes = 128 * D * kElemBytes;  // one 128 x D input tile
+  static constexpr int kOutTileBytes = 128 * D * 2;        // one 128 x D bf16 output tile
+  static constexpr int kBoxCols = 128 / kElemBytes;        // input elements per 128-byte TMA box row
+  static constexpr int kBoxes = kTileBytes / 16384;        // 128-row TMA boxes (16 KB) per input tile
+  static constexpr int kOutBoxes = D / 64;                 // 64-column bf16 boxes per output tile
+  static constexpr int kStages = (FP8 || D == 64) ? 8 : 4;  // K/V ring depth
+  // The epilogue stages O and o_lo of both query tiles in the idle ring.
+  static_assert(kStages * kTileBytes >= 4 * kOutTileBytes, "epilogue staging");
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kXOff = kKVOff + kStages * kTileBytes;  // half-row maxima [2 tiles][2 halves][128]
@@ -99,12 +110,16 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-template <int D, bool CAUSAL, bool DROPOUT = false>
+// FP8: e4m3 Q, K, V with per-head descale factors (kind::f8f6f4 MMAs, K = 32
+// per instruction); P is rounded to e4m3 for the PV product, four per TMEM
+// column, and O is divided by the fp32 row sum of the unrounded P.
+template <int D, bool CAUSAL, bool DROPOUT = false, bool FP8 = false>
 __global__ void __launch_bounds__(352, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const __grid_constant__ CUtensorMap tmOlo, const FwdParams p) {
-  using C = FwdCfg<D>;
+  static_assert(!(FP8 && DROPOUT), "no dropout in the e4m3 forward");
+  using C = FwdCfg<D, FP8>;
   extern __shared__ __align__(1024) uint8_t smem[];
 
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
@@ -197,7 +212,7 @@ __global__ void __launch_bounds__(352, 1)
       tma_prefetch_desc(&tmO);
       mbar_arrive_expect_tx(&bar_q[0], C::kTileBytes);
       for (int b = 0; b < C::kBoxes; ++b)
-        tma_load_3d(&tmQ, &bar_q[0], sQ + b * 16384, b * 64, (2 * u) * 128, bh);
+        tma_load_3d(&tmQ, &bar_q[0], sQ + b * 16384, b * C::kBoxCols, (2 * u) * 128, bh);
       int idx = 0;
       bool ok = true;
       for (; idx < 2 * n_kv && ok; ++idx) {
@@ -209,11 +224,11 @@ __global__ void __launch_bounds__(352, 1)
         uint8_t *dst = sKV + s * C::kTileBytes;
         mbar_arrive_expect_tx(&bar_kv_full[s], C::kTileBytes);
         for (int b = 0; b < C::kBoxes; ++b)
-          tma_load_3d(is_k ? &tmK : &tmV, &bar_kv_full[s], dst + b * 16384, b * 64, j * 128, bh);
+          tma_load_3d(is_k ? &tmK : &tmV, &bar_kv_full[s], dst + b * 16384, b * C::kBoxCols, j * 128, bh);
         if (idx == 0) {
           mbar_arrive_expect_tx(&bar_q[1], C::kTileBytes);
           for (int b = 0; b < C::kBoxes; ++b)
-            tma_load_3d(&tmQ, &bar_q[1], sQ + C::kTileBytes + b * 16384, b * 64, (2 * u + 1) * 128, bh);
+            tma_load_3d(&tmQ, &bar_q[1], sQ + C::kTileBytes + b * 16384, b * C::kBoxCols, (2 * u + 1) * 128, bh);
         }
       }
       if (!ok) {
@@ -231,8 +246,8 @@ __global__ void __launch_bounds__(352, 1)
     // ------------------------------------------------------------ MMA issuers
     const int k = warp - C::kIssuerWarp;  // query tile owned by this issuer
     if (lane == 0 && !*abort_flag) {
-      constexpr uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
-      constexpr uint32_t idesc_pv = make_idesc_bf16(128, D, 0, 1);
+      constexpr uint32_t idesc_qk = FP8 ? make_idesc_e4m3(128, 128, 0, 0) : make_idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t idesc_pv = FP8 ? make_idesc_e4m3(128, D, 0, 1) : make_idesc_bf16(128, D, 0, 1);
       // Base descriptors: Q_k (K-major), ring stage 0 as K (K-major) and as V (MN-major).
       const uint64_t q_desc = make_sdesc(smem_u32(sQ + k * C::kTileBytes), 16, 1024);
       const uint64_t k_desc0 = make_sdesc(smem_u32(sKV), 16, 1024);
@@ -258,10 +273,14 @@ __global__ void __launch_bounds__(352, 1)
         // this thread and the tensor pipe runs them in issue order, so S_k is
         // issued right behind PV_k without waiting for it to complete.
         const uint64_t k_desc = sdesc_add(k_desc0, sK * C::kTileBytes);
+        // One MMA per 32-byte K slice of the 128-byte swizzled rows (16 bf16 or 32 e4m3).
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
+        for (int ks = 0; ks < D * C::kElemBytes / 32; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_ss(tS, sdesc_add(q_desc, off), sdesc_add(k_desc, off), idesc_qk, ks > 0);
+          if constexpr (FP8)
+            mma_ss_f8(tS, sdesc_add(q_desc, off), sdesc_add(k_desc, off), idesc_qk, ks > 0);
+          else
+            mma_ss(tS, sdesc_add(q_desc, off), sdesc_add(k_desc, off), idesc_qk, ks > 0);
         }
         mma_commit(&bar_s_full[k]);
         mma_commit(&bar_kv_empty[sK]);
@@ -272,10 +291,19 @@ __global__ void __launch_bounds__(352, 1)
         tc_fence_after();
         FA_TRACE(16 + k * 256 + 4 * j + 2);
         const uint64_t v_desc = sdesc_add(v_desc0, sV * C::kTileBytes);
+        // K steps over the 128 keys: 16 (bf16) or 32 (e4m3) keys, 8 TMEM columns of P
+        // and 16 or 32 rows of V each; P of keys 64h.. starts at column 64h.
+        if constexpr (FP8) {
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_ts(tO, tS + ks * 8 + (ks >= 4 ? 32 : 0), sdesc_add(v_desc, ks * 2048), idesc_pv,
-                 (j > 0 || ks > 0) ? 1u : 0u);
+          for (int ks = 0; ks < 4; ++ks)
+            mma_ts_f8(tO, tS + ks * 8 + (ks >= 2 ? 48 : 0), sdesc_add(v_desc, ks * 4096), idesc_pv,
+                      (j > 0 || ks > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ts(tO, tS + ks * 8 + (ks >= 4 ? 32 : 0), sdesc_add(v_desc, ks * 2048), idesc_pv,
+                   (j > 0 || ks > 0) ? 1u : 0u);
+        }
         mma_commit(&bar_pv_done[k]);
         mma_commit(&bar_kv_empty[sV]);
         FA_TRACE(16 + k * 256 + 4 * j + 1);
@@ -294,7 +322,8 @@ __global__ void __launch_bounds__(352, 1)
     const int r = rq * 32 + lane;            // row within the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(rq * 32) << 16;
     float *xm = reinterpret_cast<float *>(smem + C::kXOff);  // [k][h][128]
-    const float c = p.scale_log2;
+    // c = scale * log2(e), times the descale factors of Q and K for e4m3 inputs.
+    const float c = FP8 ? p.scale_log2 * p.descale_q[bh] * p.descale_k[bh] : p.scale_log2;
     const uint64_t c2 = f2pack(c, c);
     float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, lr[2] = {0.f, 0.f};
     const int n_k[2] = {n_kv0, n_kv1};
@@ -348,6 +377,31 @@ __global__ void __launch_bounds__(352, 1)
         auto exps = [&](float mref) {
           const float neg = (mref == -INFINITY) ? 0.f : -mref;
           const uint64_t n2 = f2pack(neg, neg);
+          if constexpr (FP8) {
+            // P rounded to e4m3, four keys per word; O's normaliser is the fp32
+            // sum of the unrounded P (the same sum as the LSE's).
+            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+            for (int cq = 0; cq < 16; ++cq) {
+              const uint64_t xa = ffma2(f2pack(__uint_as_float(s[4 * cq]), __uint_as_float(s[4 * cq + 1])), c2, n2);
+              const uint64_t xb =
+                  ffma2(f2pack(__uint_as_float(s[4 * cq + 2]), __uint_as_float(s[4 * cq + 3])), c2, n2);
+              float x0, x1, x2, x3;
+              f2unpack(xa, x0, x1);
+              f2unpack(xb, x2, x3);
+              const float a0 = ex2(x0), a1 = ex2(x1), a2 = ex2(x2), a3 = ex2(x3);
+              acc[cq & 3] = fadd2(acc[cq & 3], fadd2(f2pack(a0, a1), f2pack(a2, a3)));
+              pk[cq] = pack_e4m3x4(a0, a1, a2, a3);
+            }
+            float u0, u1, u2, u3, u4, u5, u6, u7;
+            f2unpack(acc[0], u0, u1);
+            f2unpack(acc[1], u2, u3);
+            f2unpack(acc[2], u4, u5);
+            f2unpack(acc[3], u6, u7);
+            psum = ((u0 + u1) + (u2 + u3)) + ((u4 + u5) + (u6 + u7));
+            prsum = psum;
+            return;
+          }
           uint64_t acc[2] = {0ull, 0ull}, racc[2] = {0ull, 0ull};
 #pragma unroll
           for (int cc = 0; cc < 32; ++cc) {
@@ -402,7 +456,10 @@ __global__ void __launch_bounds__(352, 1)
             tmem_st32(tO + ch * 32, o);
           }
         }
-        tmem_st32(tS, pk);
+        if constexpr (FP8)
+          tmem_st16(tS, pk);  // 64 keys of e4m3 P in 16 columns
+        else
+          tmem_st32(tS, pk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bar_p_full[k]);
@@ -429,9 +486,9 @@ __global__ void __launch_bounds__(352, 1)
       if (r == 0 && h == 0) FA_TRACE(4 + k);
       const float lt = l[k] + ls[((h ^ 1) * 2 + 0) * 128 + r];
       const float lrt = lr[k] + ls[((h ^ 1) * 2 + 1) * 128 + r];
-      const float inv_l = (DROPOUT ? p.drop.inv_keep : 1.f) / lrt;
-      const uint32_t st_o = smem_u32(sKV + (2 * k) * C::kTileBytes);
-      const uint32_t st_lo = smem_u32(sKV + (2 * k + 1) * C::kTileBytes);
+      const float inv_l = (FP8 ? p.descale_v[bh] : (DROPOUT ? p.drop.inv_keep : 1.f)) / lrt;
+      const uint32_t st_o = smem_u32(sKV + (2 * k) * C::kOutTileBytes);
+      const uint32_t st_lo = smem_u32(sKV + (2 * k + 1) * C::kOutTileBytes);
       const uint32_t tO = tmem + lane_off + 256 + k * D;
 #pragma unroll
       for (int ch = 0; ch < D / 64; ++ch) {
@@ -474,10 +531,10 @@ __global__ void __launch_bounds__(352, 1)
         for (int k = 0; k < 2; ++k) {
           const int qt = 2 * u + k;
           if (qt * 128 >= p.N) continue;
-          for (int b = 0; b < C::kBoxes; ++b) {
-            tma_store_3d(&tmO, sKV + (2 * k) * C::kTileBytes + b * 16384, b * 64, qt * 128, bh);
+          for (int b = 0; b < C::kOutBoxes; ++b) {
+            tma_store_3d(&tmO, sKV + (2 * k) * C::kOutTileBytes + b * 16384, b * 64, qt * 128, bh);
             if (p.o_lo != nullptr)
-              tma_store_3d(&tmOlo, sKV + (2 * k + 1) * C::kTileBytes + b * 16384, b * 64, qt * 128, bh);
+              tma_store_3d(&tmOlo, sKV + (2 * k + 1) * C::kOutTileBytes + b * 16384, b * 64, qt * 128, bh);
           }
         }
         bulk_commit();

@@ -175,3 +175,30 @@ def test_selftest_without_a_device(lib):
     if torch.cuda.is_available():
         pytest.skip("a device is present")
     assert lib.fa_selftest_timeout(None) == 5
+
+
+def fwd_fp8(lib, *, q=P, dq=P, o=P, lse=P, B=1, H=2, N=256, d=128, scale=0.125, causal=0):
+    return lib.fa_fwd_fp8(q, P, P, dq, P, P, o, lse, B, H, N, d, ctypes.c_float(scale), causal, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    ({"q": None}, 1), ({"dq": None}, 1), ({"o": None}, 1), ({"lse": None}, 1), ({"N": 0}, 1),
+    ({"scale": 0.0}, 1), ({"causal": 3}, 1), ({"d": 64}, 2), ({"d": 96}, 2),
+    ({"B": 1 << 16, "H": 1 << 10, "N": 1 << 10}, 2),
+    ({"q": ctypes.c_void_p(4097)}, 3), ({"o": ctypes.c_void_p(4104)}, 3), ({"dq": ctypes.c_void_p(4098)}, 3),
+])
+def test_fp8_fwd_argument_errors(lib, kw, code):
+    """e4m3 forward: d = 128 only; 16-byte aligned tensors, 4-byte aligned descale vectors."""
+    lib.fa_fwd_fp8.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_int,
+                                                                           ctypes.c_void_p]
+    assert fwd_fp8(lib, **kw) == code
+
+
+def test_noalloc_status_calls_without_a_device(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    info = (ctypes.c_int * 4)(9, 9, 9, 9)
+    assert lib.fa_noalloc_device_status(None, info) == 5
+    assert list(info) == [0, 0, 0, 0]
+    assert lib.fa_noalloc_selftest_timeout(None) == 5

@@ -8,6 +8,9 @@ Roles, as in the kernel (one CTA: key tile j, query tiles it = 0 .. n-1):
       d = 128:  S^T(i) dP^T(i) [P^T] dV(i) [dS] dK(i) dQ(i)   (dQ in dP^T's columns,
                 so dP^T(i+1) waits until the drain has read dQ(i))
       d = 64:   S^T(0) dP^T(0) | [P^T] dV(i) S^T(i+1) [dS] dK(i) dQ(i) dP^T(i+1) | ...
+      no dQ (the deterministic mode's instantiation, both d):
+                S^T(0) dP^T(0) | [P^T] dV(i) S^T(i+1) [dS] dK(i) dP^T(i+1) | ...
+                with dK(i) committing what dQ(i) commits otherwise;
     S^T(i+1) is put in behind dV(i), which reads P^T(i) from the same columns;
   * eight compute warps (query-column half w, key-row quarter q): read their part
     of S^T, write P^T over it, then read their part of dP^T and write their rows
@@ -17,7 +20,7 @@ Roles, as in the kernel (one CTA: key tile j, query tiles it = 0 .. n-1):
   * four dQ drain warps: read their rows of dQ out of TMEM (then the issuer may
     reuse the columns), stage them in tile it's Q / dO stage buffers, and the
     leader reduce-adds them into the accumulator and hands the stage back to the
-    producer;
+    producer (without dQ, the leader only hands the stage back);
   * epilogue: after the last dK / dQ and the drain, dV and dK are staged in the
     stage-0 buffers and stored.
 Checked: no deadlock or phase aliasing; every MMA reads the intended tiles;
@@ -38,7 +41,7 @@ def parts(name):
     return [(name, w, q) for w in HALVES for q in QUARTERS]
 
 
-def bwd_model(n_it: int, d: int, seed: int, dropout: bool = False, skip: str = "") -> None:
+def bwd_model(n_it: int, d: int, seed: int, dropout: bool = False, skip: str = "", no_dq: bool = False) -> None:
     M = Machine(seed)
     bar_kv = Bar("kv", 2)
     qdo_full = [Bar(f"qdo_full{s}", 4) for s in range(2)]  # Q, dO, LSE, D
@@ -82,6 +85,8 @@ def bwd_model(n_it: int, d: int, seed: int, dropout: bool = False, skip: str = "
         def dK(it):
             s = it & 1
             M.mma(0, {**{p: ("dS", it) for p in parts("dS")}, ("Q", s): ("Q", it), "dK": it}, {"dK": it + 1})
+            if no_dq:  # without the dQ product, dK(i) closes the tile
+                M.commit(0, dkq_done)
 
         def dQ(it):
             cols = parts(dq_cols) if d == 128 else [(dq_cols, 0, q) for q in QUARTERS]
@@ -89,7 +94,23 @@ def bwd_model(n_it: int, d: int, seed: int, dropout: bool = False, skip: str = "
             M.commit(0, dkq_done)
 
         yield lambda: bar_kv.ready(0)
-        if d == 128:
+        if no_dq:
+            # S^T(0) dP^T(0) | dV(i) S^T(i+1) [dS] dK(i) dP^T(i+1) | ... at both d
+            yield stage_ready(0)
+            sT(0)
+            dPT(0)
+            for it in range(n_it):
+                yield lambda it=it: p_full.ready(it)
+                dV(it)
+                if it + 1 < n_it:
+                    yield stage_ready(it + 1)
+                    sT(it + 1)
+                if skip != "ds_wait":
+                    yield lambda it=it: ds_full.ready(it)
+                dK(it)
+                if it + 1 < n_it:
+                    dPT(it + 1)
+        elif d == 128:
             for it in range(n_it):
                 yield stage_ready(it)
                 sT(it)
@@ -152,6 +173,14 @@ def bwd_model(n_it: int, d: int, seed: int, dropout: bool = False, skip: str = "
             M.read(("dO", 0), "dK staged")
 
     def drain(q):
+        if no_dq:  # the leader only hands each stage back once its MMAs completed
+            if q == 0:
+                for it in range(n_it):
+                    yield lambda it=it: dkq_done.ready(it)
+                    qdo_empty[it & 1].arrive()
+                    if it == n_it - 1:
+                        drained.arrive()
+            return
         for it in range(n_it):
             s = it & 1
             yield lambda it=it: dkq_done.ready(it)
@@ -183,6 +212,24 @@ def bwd_model(n_it: int, d: int, seed: int, dropout: bool = False, skip: str = "
 def test_pipeline_under_random_interleavings(n_it, d, dropout):
     for seed in range(40):
         bwd_model(n_it, d, seed, dropout=dropout)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("n_it", [1, 2, 3, 5, 8])
+def test_no_dq_pipeline_under_random_interleavings(n_it, d):
+    """The deterministic mode's instantiation: no dQ product, no dQ drain."""
+    for seed in range(40):
+        bwd_model(n_it, d, seed, no_dq=True)
+
+
+def test_no_dq_model_detects_a_missing_wait():
+    failures = 0
+    for seed in range(40):
+        try:
+            bwd_model(4, 128, seed, no_dq=True, skip="ds_wait")
+        except AssertionError:
+            failures += 1
+    assert failures > 0
 
 
 @pytest.mark.parametrize("d,dropout,skip", [(128, False, "ds_wait"), (64, True, "draws_wait")])

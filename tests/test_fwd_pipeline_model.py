@@ -160,7 +160,7 @@ CASES = [(1, 0, False), (1, 0, True), (2, 0, True), (3, 1, True), (4, 1, True), 
          (9, 4, True), (6, 2, False)]
 
 
-@pytest.mark.parametrize("stages", [4, 8])  # the kernel's ring at d = 128 and d = 64
+@pytest.mark.parametrize("stages", [4, 8])  # the kernel's ring: bf16 at d = 128; d = 64 and e4m3
 @pytest.mark.parametrize("n_all,u,causal", CASES, ids=lambda x: str(x))
 def test_pipeline_under_random_interleavings(n_all, u, causal, stages):
     n_k = tiles(n_all, u, causal)
@@ -184,5 +184,5 @@ def test_model_rings_match_the_kernel():
     import os
     import re
     src = open(os.path.join(os.path.dirname(__file__), "..", "io_aware_exact_23_b200", "csrc", "fa_fwd.cuh")).read()
-    m = re.search(r"kStages = \(D == 128\) \? (\d+) : (\d+);", src)
+    m = re.search(r"kStages = \(FP8 \|\| D == 64\) \? (\d+) : (\d+);", src)
     assert m and {int(m.group(1)), int(m.group(2))} == {4, 8}
