@@ -57,7 +57,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference", "vanilla"], default="ours")
     ap.add_argument("--workload", default="b2h32n4096d128_causal")
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget-s", type=float, default=12.0,
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -729,38 +729,64 @@ def main():
         [ms, fwd_ms, bwd_ms, main_ms, pre_ms, conv_ms, float(status)], dist, dev)
 
     # ---------------------------------------------------------------- e2e
+    # The same step from pinned host memory and back, every step: copy the step's
+    # Q, K, V, dO in, run fa_fwd + fa_bwd through the C ABI, copy O, LSE, dQ, dK,
+    # dV out.  Two device buffer sets and three streams (copy-in, compute,
+    # copy-out) ordered by events let step t's compute overlap step t+1's
+    # inputs and step t-1's outputs; every step's copies are inside the timed
+    # region, which ends when the last step's outputs have reached the host.
     e2e = None
     if args.e2e_steps > 0:
-        pin = {nm: t[nm].cpu().pin_memory() for nm in ("q", "k", "v", "do")}
-        out_h = {"o": torch.empty(o.shape, dtype=o.dtype, pin_memory=True),
-                 "lse": torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True),
-                 "dq": torch.empty(dq.shape, dtype=dq.dtype, pin_memory=True),
-                 "dk": torch.empty(dk.shape, dtype=dk.dtype, pin_memory=True),
-                 "dv": torch.empty(dv.shape, dtype=dv.dtype, pin_memory=True)}
+        names_in, names_out = ("q", "k", "v", "do"), ("o", "lse", "dq", "dk", "dv")
+        pin = {nm: t[nm].cpu().pin_memory() for nm in names_in}
+        dev_sets = [{"q": q, "k": k, "v": v, "do": dO, "o": o, "o_lo": o_lo, "lse": lse, "dq": dq, "dk": dk,
+                     "dv": dv, "ws": ws}]
+        dev_sets.append({nm: torch.empty_like(x) for nm, x in dev_sets[0].items()})
+        host_out = [{nm: torch.empty(dev_sets[0][nm].shape, dtype=dev_sets[0][nm].dtype, pin_memory=True)
+                     for nm in names_out} for _ in range(2)]
         h2d = sum(x.numel() * x.element_size() for x in pin.values())
-        d2h = sum(x.numel() * x.element_size() for x in out_h.values())
+        d2h = sum(x.numel() * x.element_size() for x in host_out[0].values())
+        s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        E = args.e2e_steps
+        ev_in = [torch.cuda.Event() for _ in range(E)]
+        ev_comp = [torch.cuda.Event() for _ in range(E)]
+        ev_out = [torch.cuda.Event() for _ in range(E)]
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         e0, e1 = mk(), mk()
-        e0.record()
-        for _ in range(args.e2e_steps):
-            q.copy_(pin["q"], non_blocking=True)
-            k.copy_(pin["k"], non_blocking=True)
-            v.copy_(pin["v"], non_blocking=True)
-            dO.copy_(pin["do"], non_blocking=True)
-            step()
-            out_h["o"].copy_(o, non_blocking=True)
-            out_h["lse"].copy_(lse, non_blocking=True)
-            out_h["dq"].copy_(dq, non_blocking=True)
-            out_h["dk"].copy_(dk, non_blocking=True)
-            out_h["dv"].copy_(dv, non_blocking=True)
-        e1.record()
+        e0.record(s_in)
+        for st in range(E):
+            D, Hh = dev_sets[st % 2], host_out[st % 2]
+            with torch.cuda.stream(s_in):
+                if st >= 2:
+                    s_in.wait_event(ev_comp[st - 2])  # set st % 2's inputs were consumed
+                for nm in names_in:
+                    D[nm].copy_(pin[nm], non_blocking=True)
+                ev_in[st].record(s_in)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(ev_in[st])
+                if st >= 2:
+                    s_comp.wait_event(ev_out[st - 2])  # set st % 2's outputs reached the host
+                fa.fa_fwd(D["q"], D["k"], D["v"], D["o"], D["lse"], w.scale, w.causal, o_lo=D["o_lo"])
+                fa.fa_bwd(D["q"], D["k"], D["v"], D["o"], D["do"], D["lse"], D["dq"], D["dk"], D["dv"], w.scale,
+                          w.causal, D["ws"], o_lo=D["o_lo"])
+                ev_comp[st].record(s_comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[st])
+                for nm in names_out:
+                    Hh[nm].copy_(D[nm], non_blocking=True)
+                ev_out[st].record(s_out)
+        s_in.wait_stream(s_out)
+        e1.record(s_in)
         torch.cuda.synchronize()
-        e2e_ms = reduce_max([e0.elapsed_time(e1) / args.e2e_steps], dist, dev)[0]
+        if fa.fa_device_status() != 0:
+            raise SystemExit("bench.py: device status error in the e2e leg")
+        e2e_ms = reduce_max([e0.elapsed_time(e1) / E], dist, dev)[0]
         e2e = {"value": world * (w.fwd_flops() + w.bwd_flops()) / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-               "path": "pinned host -> device copies, fa_fwd + fa_bwd through the C ABI, outputs -> pinned host"}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": E,
+               "path": "pinned host -> device copies, fa_fwd + fa_bwd through the C ABI, outputs -> pinned host; "
+                       "two buffer sets, copy-in / compute / copy-out streams overlapped across steps"}
 
     if rank == 0:
         peaks, peak_kind = load_peaks()
