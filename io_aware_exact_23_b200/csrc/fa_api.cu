@@ -57,10 +57,64 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
+// Tensor maps are pure functions of (address, type, dims, box), so encoded maps
+// are kept in a small least-recently-used cache: a call on tensors seen before
+// copies its maps instead of encoding them again.
+struct MapKey {
+  int dev;
+  const void *ptr;
+  int dt, D, N, BH, box_x;
+  bool operator==(const MapKey &o) const {
+    return dev == o.dev && ptr == o.ptr && dt == o.dt && D == o.D && N == o.N && BH == o.BH && box_x == o.box_x;
+  }
+};
+struct MapSlot {
+  MapKey key;
+  CUtensorMap map;
+  uint64_t used = 0;  // 0: empty
+};
+constexpr int kMapSlots = 64;
+std::mutex g_map_mu;
+MapSlot g_maps[kMapSlots];
+uint64_t g_map_tick = 0;
+
+int encode_3d_uncached(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int elem_bytes, int D, int N,
+                       int BH, int box_x);
+
 // [BH, N, D] tensor viewed as 3-D (x = feature, y = row, z = head); box of
-// 64 (or 32 for fp32) features x 128 rows x 1 head, 128-byte swizzle, zero fill.
+// 64 (or 32 for fp32, 128 for bytes) features x 128 rows x 1 head, 128-byte
+// swizzle, zero fill.
 int encode_3d(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int elem_bytes, int D, int N, int BH,
               int box_x) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  const MapKey key{dev, ptr, static_cast<int>(dt), D, N, BH, box_x};
+  {
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    for (MapSlot &sl : g_maps)
+      if (sl.used != 0 && sl.key == key) {
+        sl.used = ++g_map_tick;
+        *m = sl.map;
+        return FA_OK;
+      }
+  }
+  const int st = encode_3d_uncached(m, ptr, dt, elem_bytes, D, N, BH, box_x);
+  if (st != FA_OK) return st;
+  std::lock_guard<std::mutex> lock(g_map_mu);
+  MapSlot *victim = &g_maps[0];
+  for (MapSlot &sl : g_maps)
+    if (sl.used < victim->used) victim = &sl;
+  victim->key = key;
+  victim->map = *m;
+  victim->used = ++g_map_tick;
+  return FA_OK;
+}
+
+int encode_3d_uncached(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int elem_bytes, int D, int N,
+                       int BH, int box_x) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return FA_ERR_CUDA;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};

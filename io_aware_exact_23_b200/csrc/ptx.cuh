@@ -118,36 +118,6 @@ __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
   }
 }
 
-// ------------------------------------------------- cluster launch control
-// Ask the hardware to cancel the launch of a CTA of this grid that has not
-// started yet; the 16-byte response lands in `resp` (shared, 16-byte aligned)
-// and completes 16 transaction bytes on `bar`.  Used by persistent CTAs to take
-// over the work of CTAs that never launch.  After a response that reports no
-// cancellation, no further request may be made.
-__device__ __forceinline__ void clc_try_cancel(void *resp, uint64_t *bar) {
-  asm volatile(
-      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];" ::"r"(
-          smem_u32(resp)),
-      "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Decode a try_cancel response: the x index of the cancelled CTA, or -1 when
-// nothing was cancelled (every CTA of the grid has launched).
-__device__ __forceinline__ int clc_decode(const void *resp) {
-  uint32_t ok, x = 0;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b128 r;\n\t"
-      "ld.shared.b128 r, [%2];\n\t"
-      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t"
-      "@p clusterlaunchcontrol.query_cancel.get_first_ctaid.v4.b32.b128 {%1, _, _, _}, r;\n\t}"
-      : "=r"(ok), "+r"(x)
-      : "r"(smem_u32(resp))
-      : "memory");
-  return ok ? static_cast<int>(x) : -1;
-}
-
 // ------------------------------------------------------------------ fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
