@@ -202,3 +202,14 @@ def test_noalloc_status_calls_without_a_device(lib):
     assert lib.fa_noalloc_device_status(None, info) == 5
     assert list(info) == [0, 0, 0, 0]
     assert lib.fa_noalloc_selftest_timeout(None) == 5
+
+
+def test_element_limit_is_exact(lib):
+    """Tensors of up to 2^31 - 1 elements are accepted; one more row is refused."""
+    f = lib.fa_bwd_workspace_bytes
+    f.restype = ctypes.c_size_t
+    for B, H, d in [(1, 1, 128), (1, 16, 128), (2, 32, 64)]:
+        n_max = (2 ** 31 - 1) // (B * H * d)
+        assert f(B, H, n_max, d) > 0
+        assert f(B, H, n_max + 1, d) == 0
+        assert fwd(lib, B=B, H=H, N=n_max + 1, d=d) == 2

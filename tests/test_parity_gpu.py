@@ -223,3 +223,36 @@ SWEEP = I.sweep()
 @pytest.mark.parametrize("w", SWEEP, ids=lambda w: w.name)
 def test_sweep_point(w):
     check_sampled(w, n_rows=64, dkdv_full_head_max_n=1024)
+
+
+@pytest.mark.slow
+def test_very_long_sequence_sampled():
+    """B=1, H=1, N=262144, d=128, causal: 64x the long-context workload's tokens
+    per head.  O, LSE and dQ at sampled rows (first, tile edges, middle, last)
+    against the oracle, dK / dV element by element on the last key tile (whose
+    query statistics are cheap to get at this N), and the gradient identities
+    over the whole head."""
+    w = Workload("very_long_b1h1n262144d128_causal", 1, 1, 262144, 128, True, seed=17)
+    t = make_inputs(w, device="cuda")
+    o, lse, o_lo = gpu_forward(t, w.scale, True, residual=True)
+    dq, dk, dv = gpu_backward(t, o, lse, w.scale, True, o_lo=o_lo)
+    N, d = w.N, w.d
+    sb, sr = sample_rows(1, N, 24, seed=N)
+    o_ref, l_ref = oracle.ref_fwd_rows(t["q"], t["k"], t["v"], w.scale, True, sb, sr)
+    of, lf = to64(o).reshape(N, d), to64(lse).reshape(N)
+    assert max_err(of[sr], o_ref) <= TOL_O
+    assert max_err(lf[sr], l_ref) <= TOL_LSE
+    dq_ref = oracle.ref_dq_rows(t["q"], t["k"], t["v"], t["do"], w.scale, True, sb, sr)
+    assert max_err(to64(dq).reshape(N, d)[sr], dq_ref) <= TOL_GRAD_REL * np.abs(dq_ref).max()
+    keys = np.arange(N - 128, N)
+    rk, rv = oracle.ref_dkdv_rows(t["q"], t["k"], t["v"], t["do"], w.scale, True, 0, keys)
+    for g, r in ((to64(dk).reshape(N, d)[keys], rk), (to64(dv).reshape(N, d)[keys], rv)):
+        assert max_err(g, r) <= TOL_GRAD_REL * np.abs(r).max()
+    dk64, dv64, dq64 = dk.double(), dv.double(), dq.double()
+    assert (dk64.sum(2).abs().amax() <= TOL_GRAD_REL * dk64.abs().amax() * np.sqrt(N) + 1e-6).all()
+    s_dv = (dv64.sum(2) - t["do"].double().sum(2)).abs().amax()
+    assert s_dv <= TOL_GRAD_REL * dv64.abs().amax() * np.sqrt(N) + 1e-6
+    lhs = (t["q"].double() * dq64).sum()
+    rhs = (t["k"].double() * dk64).sum()
+    mag = (t["q"].double().abs() * dq64.abs()).sum() + (t["k"].double().abs() * dk64.abs()).sum()
+    assert (lhs - rhs).abs() <= TOL_GRAD_REL * mag
