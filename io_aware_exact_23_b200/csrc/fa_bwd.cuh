@@ -18,16 +18,19 @@
 //                          contribution is added into the fp32 accumulator.
 //   3. fa_dq_convert_kernel  dQ (bf16) = accumulator.
 //
-// fa_bwd_kernel roles (448 threads):
+// fa_bwd_kernel roles (448 threads at d = 64; 320 at d = 128 and without dQ):
 //   warps 0-3   compute, query columns 0..63 of each tile (thread = key row)
 //   warps 4-7   compute, query columns 64..127
-//   warps 8-11  dQ drain: TMEM dQ rows -> registers (TMEM released at once) ->
-//               scale -> the Q_i / dO_i stage buffers of the finished tile
-//               (together exactly one fp32 dQ tile) -> TMA bulk reduce-add into
-//               the fp32 accumulator in L2; the drain then hands the stage back
-//               to the producer
-//   warp  12    TMA producer: K_j, V_j once; Q_i, dO_i, LSE_i, D_i per tile (2 stages)
-//   warp  13    MMA issuer (one thread), five MMAs per query tile:
+//   dQ drain    TMEM dQ rows -> registers (TMEM released at once) -> scale ->
+//               the Q_i / dO_i stage buffers of the finished tile (together
+//               exactly one fp32 dQ tile) -> TMA bulk reduce-add into the fp32
+//               accumulator in L2, then the stage goes back to the producer.
+//               At d = 64 four warps (8-11) do it, their leader issuing the
+//               reduce-add; at d = 128 the compute warps stage dQ themselves
+//               after each tile's dS and the producer issues the reduce-add.
+//   producer    (warp 12 / 8) TMA: K_j, V_j once; Q_i, dO_i, LSE_i, D_i per
+//               tile (2 stages)
+//   issuer      (warp 13 / 9) MMAs (one thread), five per query tile:
 //                 S^T  = K_j Q_i^T      (smem x smem)      -> TMEM
 //                 dP^T = V_j dO_i^T     (smem x smem)      -> TMEM
 //                 dV  += P^T dO_i       (TMEM x smem)
@@ -91,9 +94,22 @@ struct BwdCfg {
   static constexpr int kNumBars = 17;  // then the TMEM address slot and the abort flag
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static constexpr int kThreads = 448;
   static constexpr uint32_t kColS = 0, kColdP = 128, kColdK = 256, kColdV = 256 + D;
   static constexpr uint32_t kColdQ = (D == 128) ? 128 : 384;
+};
+
+// Warp roles.  With the dQ product at d = 64 there are four drain warps (8-11)
+// that stage each tile's dQ for the reduce-add.  At d = 128 the compute warps
+// drain dQ themselves, in the time they would otherwise spend waiting for dK,
+// dQ and the next S^T, and the producer reduce-adds the staged tile just before
+// it reloads that stage; without the dQ product (the deterministic mode) there
+// is nothing to drain.  Either way ten warps, and up to 168 registers a thread.
+template <int D, bool NO_DQ>
+struct BwdRoles {
+  static constexpr bool kComputeDrain = (D == 128) || NO_DQ;
+  static constexpr int kThreads = kComputeDrain ? 320 : 448;
+  static constexpr int kProducerWarp = kComputeDrain ? 8 : 12;
+  static constexpr int kIssuerWarp = kComputeDrain ? 9 : 13;
 };
 
 enum BwdTag : int {
@@ -203,20 +219,22 @@ __global__ void __launch_bounds__(256) fa_dq_convert_kernel(const float *__restr
 // fa_dq_kernel.  It skips the dQ product and its drain; dK(i) then closes each
 // query tile (its commit takes the place of dQ(i)'s), the issue order is
 // S^T(0) dP^T(0) | dV(i) S^T(i+1) dK(i) dP^T(i+1) | ... at both head dims, and
-// the drain warps' leader only hands each Q_i / dO_i stage back to the producer.
+// the producer reloads each Q_i / dO_i stage once dK(i) has completed.
 template <int D, bool CAUSAL, bool DROPOUT = false, bool NO_DQ = false>
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                   const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
                   const __grid_constant__ CUtensorMap tmdQacc, const BwdParams p) {
   using C = BwdCfg<D>;
+  using R = BwdRoles<D, NO_DQ>;
   extern __shared__ __align__(1024) uint8_t smem[];
 
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
   uint64_t *bar_kv = bars + 0;
   uint64_t *bar_qdo_full = bars + 1;   // [2]
-  uint64_t *bar_qdo_empty = bars + 3;  // [2]
+  uint64_t *bar_qdo_empty = bars + 3;  // [2] drain-warp layout: the stage is free again
+  uint64_t *bar_staged = bars + 3;     // [2] compute-drain layout: every compute thread staged its dQ part
   uint64_t *bar_s_full = bars + 5;
   uint64_t *bar_dp_full = bars + 6;
   uint64_t *bar_p_full = bars + 7;
@@ -256,7 +274,7 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(bar_kv, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar_qdo_full[s], 1);
-      mbar_init(&bar_qdo_empty[s], 1);
+      mbar_init(&bar_qdo_empty[s], R::kComputeDrain ? 256 : 1);  // bar_staged in that layout
     }
     mbar_init(bar_s_full, 1);
     mbar_init(bar_dp_full, 1);
@@ -264,7 +282,7 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(bar_ds_full, 256);
     mbar_init(bar_spare, 1);
     mbar_init(bar_dkq_done, 1);
-    mbar_init(bar_dq_empty, 128);
+    mbar_init(bar_dq_empty, R::kComputeDrain ? 256 : 128);
     mbar_init(bar_epi, 256);
     mbar_init(bar_drain, 1);
     mbar_init(bar_drained, 1);
@@ -273,7 +291,7 @@ __global__ void __launch_bounds__(448, 1)
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == 13) {
+  if (warp == R::kIssuerWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -283,7 +301,7 @@ __global__ void __launch_bounds__(448, 1)
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) FA_TRACE(0);
 
-  if (warp == 12) {
+  if (warp == R::kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && !*abort_flag) {
       tma_prefetch_desc(&tmQ);
@@ -297,9 +315,35 @@ __global__ void __launch_bounds__(448, 1)
       }
       bool ok = true;
       int it = 0;
+      // Compute-drain layout: query tile t's stage is reloaded (for tile t + 2)
+      // once the tile is done with -- after dK(t)'s commit without the dQ
+      // product (dK(t+1) is issued behind S^T(t+2), which needs this reload, so
+      // the parity wait cannot fall two phases behind); else once every compute
+      // thread has staged its part of dQ(t) there and this thread has
+      // reduce-added the staged tile into the accumulator (and TMA has read it).
+      auto free_stage = [&](int t) -> bool {
+        const int st = t & 1;
+        if constexpr (NO_DQ) {
+          return mbar_wait(ctx, bar_dkq_done, t & 1, kBTagDkqDone);
+        } else {
+          if (!mbar_wait(ctx, &bar_staged[st], (t >> 1) & 1, kBTagStage)) return false;
+          for (int half = 0; half < 2; ++half)
+            for (int b = 0; b < D / 64; ++b)
+              tma_reduce_add_3d(&tmdQacc, (half == 0 ? sQ : sdO) + st * C::kTile + b * 16384,
+                                half * (D / 2) + 32 * b, (i0 + t) * 128, bh);
+          bulk_commit();
+          bulk_wait_read<0>();
+          return true;
+        }
+      };
       for (; it < n_it; ++it) {
         const int s = it & 1, n = it >> 1;
-        if (n > 0 && !mbar_wait(ctx, &bar_qdo_empty[s], (n - 1) & 1, kBTagQdoEmpty)) {
+        if constexpr (R::kComputeDrain) {
+          if (it >= 2 && !free_stage(it - 2)) {
+            ok = false;
+            break;
+          }
+        } else if (n > 0 && !mbar_wait(ctx, &bar_qdo_empty[s], (n - 1) & 1, kBTagQdoEmpty)) {
           ok = false;
           break;
         }
@@ -313,6 +357,17 @@ __global__ void __launch_bounds__(448, 1)
         bulk_load_1d(sL + s * 128, p.ws_lse2 + soff, 512, &bar_qdo_full[s]);
         bulk_load_1d(sDv + s * 128, p.ws_D + soff, 512, &bar_qdo_full[s]);
       }
+      if constexpr (R::kComputeDrain) {
+        // The last two tiles have no load behind them: reduce-add their staged dQ
+        // here, then let the epilogue have the stage buffers.  Without the dQ
+        // product there is nothing to wait for: the epilogue waits for the last
+        // dK itself, and a wait here for dK(n-2) could miss its phase -- dK(n-1)
+        // does not depend on this thread, so it may complete first.
+        if constexpr (!NO_DQ)
+          for (int t = n_it >= 2 ? n_it - 2 : 0; t < n_it && ok; ++t) ok = free_stage(t);
+        if (ok) mbar_arrive(bar_drained);
+        if constexpr (!NO_DQ) bulk_wait<0>();  // every reduction has landed before the CTA exits
+      }
       if (!ok) {
         mbar_drain(bar_kv, 0);
         for (int s = 0; s < 2 && s < it; ++s) {
@@ -322,7 +377,7 @@ __global__ void __launch_bounds__(448, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 13) {
+  } else if (warp == R::kIssuerWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && !*abort_flag) {
       constexpr uint32_t id_ss = make_idesc_bf16(128, 128, 0, 0);     // S^T, dP^T
@@ -577,6 +632,37 @@ __global__ void __launch_bounds__(448, 1)
       tc_fence_before();
       mbar_arrive(bar_ds_full);
       if (threadIdx.x == 0) FA_TRACE(16 + it * 8 + 7);
+      if constexpr (R::kComputeDrain && !NO_DQ) {
+        // dQ drain: once dK(i) and dQ(i) have completed, read this warp's part of
+        // dQ (its lane quarter's rows, columns 64w..) out of TMEM -- which frees
+        // the columns for dP^T(i+1) -- and stage it, scaled, as fp32 in tile i's
+        // Q (w = 0) or dO (w = 1) stage buffer for the producer's reduce-add.
+        ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, it & 1, kBTagDkqDone));
+        if (!ok) break;
+        tc_fence_after();
+        if (threadIdx.x == 0) FA_TRACE(1024 + it * 2 + 0);
+        uint32_t v[64];
+        const uint32_t tdQ = tmem + lane_off + C::kColdQ + 64 * w;
+        tmem_ld32(tdQ, v);
+        tmem_ld32(tdQ + 32, v + 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar_dq_empty);
+        const uint32_t buf = smem_u32((w == 0 ? sQ : sdO) + s * C::kTile);
+#pragma unroll
+        for (int b = 0; b < 2; ++b)
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int c0 = 32 * b + 4 * t;
+            st_shared_v4(buf + b * 16384 + bsw128(r, t), __float_as_uint(__uint_as_float(v[c0]) * p.scale),
+                         __float_as_uint(__uint_as_float(v[c0 + 1]) * p.scale),
+                         __float_as_uint(__uint_as_float(v[c0 + 2]) * p.scale),
+                         __float_as_uint(__uint_as_float(v[c0 + 3]) * p.scale));
+          }
+        fence_proxy_async_smem();
+        mbar_arrive(&bar_staged[s]);
+        if (threadIdx.x == 0) FA_TRACE(1024 + it * 2 + 1);
+      }
     }
     // ---------------------------------------------------------- epilogue
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, (n_it - 1) & 1, kBTagDkqDone) &&
@@ -623,21 +709,7 @@ __global__ void __launch_bounds__(448, 1)
       }
     }
     __syncwarp();
-  } else if (NO_DQ) {
-    // --------------------------------------- stage release (no dQ to drain)
-    // The stage of query tile it is free once every MMA issued up to dK(it) --
-    // among them the four that read Q_i and dO_i -- has completed.
-    if (warp == 8 && lane == 0) {
-      bool ok = !*abort_flag;
-      for (int it = 0; it < n_it && ok; ++it) {
-        ok = mbar_wait(ctx, bar_dkq_done, it & 1, kBTagDkqDone);
-        if (!ok) break;
-        mbar_arrive(&bar_qdo_empty[it & 1]);
-        if (it == n_it - 1) mbar_arrive(bar_drained);
-      }
-    }
-    __syncwarp();
-  } else {
+  } else if constexpr (!R::kComputeDrain) {
     // ------------------------------------------------------------ dQ drain
     // Staging: the fp32 dQ tile is 128 rows x D columns = 4 * D * 128 bytes, split
     // into 32-column boxes (128-byte swizzle); boxes 0..D/64-1 go to Q_i's stage
@@ -704,7 +776,7 @@ __global__ void __launch_bounds__(448, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 13) tmem_dealloc(tmem, 512);
+  if (warp == R::kIssuerWarp) tmem_dealloc(tmem, 512);
 }
 
 // ------------------------------------------------------------ host side
@@ -753,7 +825,7 @@ inline cudaError_t bwd_set_attributes() {
 template <int D, bool CAUSAL, bool DROPOUT, bool NO_DQ = false>
 inline void bwd_main_launch(const CUtensorMap *m, const BwdParams &p, int nkv, cudaStream_t s) {
   const dim3 grid(static_cast<unsigned>(p.BH) * static_cast<unsigned>(nkv));
-  fa_bwd_kernel<D, CAUSAL, DROPOUT, NO_DQ><<<grid, BwdCfg<D>::kThreads, BwdCfg<D>::kSmemBytes, s>>>(
+  fa_bwd_kernel<D, CAUSAL, DROPOUT, NO_DQ><<<grid, BwdRoles<D, NO_DQ>::kThreads, BwdCfg<D>::kSmemBytes, s>>>(
       m[0], m[1], m[2], m[3], m[4], m[5], m[6], p);
 }
 

@@ -25,6 +25,9 @@ what is in flight:
   or load using the buffer in flight.
 * A role yields a predicate to wait on (``lambda: True`` to just yield), and
   is resumed only when the predicate holds.
+* Scheduling: each run picks one role (or none) to be slow -- while it is ready
+  it is chosen 50 times less often than any other event -- so that runs also
+  explore a waiter that falls far behind the barriers it waits on.
 
 ``Machine.run`` fails on a deadlock (no role, load or MMA can make progress
 before every role has finished) and on any failed check.
@@ -103,6 +106,7 @@ class Machine:
     def run(self, roles, max_events: int = 400000):
         waits = [None] * len(roles)
         done = [False] * len(roles)
+        slow = self.rnd.randrange(len(roles) + 1)  # len(roles): no slow role
         for _ in range(max_events):
             opts = [("role", a) for a in range(len(roles)) if not done[a] and (waits[a] is None or waits[a]())]
             if self.loads:
@@ -113,7 +117,7 @@ class Machine:
             if not opts:
                 assert all(done), f"deadlock: roles finished {done}"
                 return
-            op = self.rnd.choice(opts)
+            op = self.rnd.choices(opts, weights=[0.02 if o == ("role", slow) else 1.0 for o in opts])[0]
             if op[0] == "role":
                 a = op[1]
                 try:

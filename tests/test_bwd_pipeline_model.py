@@ -3,7 +3,11 @@ interleavings (engine: tests/pipeline_model.py).
 
 Roles, as in the kernel (one CTA: key tile j, query tiles it = 0 .. n-1):
   * producer: K_j and V_j once; per query tile Q_i, dO_i, LSE_i, D_i into stage
-    it % 2, each stage after its "empty" barrier;
+    it % 2.  With drain warps (d = 64) it reloads a stage after its "empty"
+    barrier; in the compute-drain layout (d = 128, and every no-dQ instantiation)
+    it frees tile i - 2's stage itself just before reloading it: it waits for the
+    compute warps' staged dQ(i-2) and reduce-adds it (no dQ: it waits for
+    dK(i-2)), and frees the last two tiles the same way after the last load;
   * issuer (one thread), five MMAs per query tile:
       d = 128:  S^T(i) dP^T(i) [P^T] dV(i) [dS] dK(i) dQ(i)   (dQ in dP^T's columns,
                 so dP^T(i+1) waits until the drain has read dQ(i))
@@ -16,11 +20,13 @@ Roles, as in the kernel (one CTA: key tile j, query tiles it = 0 .. n-1):
     of S^T, write P^T over it, then read their part of dP^T and write their rows
     of the dS tile in shared memory (after the previous tile's dK / dQ, which
     read it, have completed).  With dropout they first stage the generator's
-    draws in their own part of the dS tile (after the same wait);
-  * four dQ drain warps: read their rows of dQ out of TMEM (then the issuer may
-    reuse the columns), stage them in tile it's Q / dO stage buffers, and the
-    leader reduce-adds them into the accumulator and hands the stage back to the
-    producer (without dQ, the leader only hands the stage back);
+    draws in their own part of the dS tile (after the same wait).  At d = 128
+    they then drain dQ: once dK(i) and dQ(i) completed, read their part of dQ
+    out of TMEM (then the issuer may reuse the columns) and stage it in tile i's
+    Q (w = 0) or dO (w = 1) stage buffer;
+  * d = 64 only, four dQ drain warps: read their rows of dQ out of TMEM, stage
+    them in tile it's Q / dO stage buffers, and the leader reduce-adds them into
+    the accumulator and hands the stage back to the producer;
   * epilogue: after the last dK / dQ and the drain, dV and dK are staged in the
     stage-0 buffers and stored.
 Checked: no deadlock or phase aliasing; every MMA reads the intended tiles;
@@ -43,15 +49,28 @@ def parts(name):
 
 def bwd_model(n_it: int, d: int, seed: int, dropout: bool = False, skip: str = "", no_dq: bool = False) -> None:
     M = Machine(seed)
+    compute_drain = d == 128 or no_dq  # the kernel's BwdRoles::kComputeDrain
     bar_kv = Bar("kv", 2)
     qdo_full = [Bar(f"qdo_full{s}", 4) for s in range(2)]  # Q, dO, LSE, D
     qdo_empty = [Bar(f"qdo_empty{s}", 1) for s in range(2)]
+    staged = [Bar(f"staged{s}", 8) for s in range(2)]  # compute-drain layout
     s_full, dp_full = Bar("s_full", 1), Bar("dp_full", 1)
     p_full, ds_full = Bar("p_full", 8), Bar("ds_full", 8)
-    dkq_done, dq_empty = Bar("dkq_done", 1), Bar("dq_empty", 4)
+    dkq_done, dq_empty = Bar("dkq_done", 1), Bar("dq_empty", 8 if compute_drain else 4)
     epi, drained, stage = Bar("epi", 8), Bar("drained", 1), Bar("stage", 4)
     M.tag["dK"] = M.tag["dV"] = 0
     dq_cols = "dPT" if d == 128 else "dQc"  # dQ's TMEM columns
+
+    def free_stage(t):
+        """Compute-drain layout: the producer frees tile t's stage."""
+        st = t & 1
+        if no_dq:
+            yield lambda: dkq_done.ready(t)
+            return
+        if skip != "staged_wait":
+            yield lambda: staged[st].ready(t >> 1)
+        M.read(("Q", st), ("dQ staged", t))  # the reduce-add's read (waited for)
+        M.read(("dO", st), ("dQ staged", t))
 
     def producer():
         yield lambda: True
@@ -59,10 +78,18 @@ def bwd_model(n_it: int, d: int, seed: int, dropout: bool = False, skip: str = "
         M.load("V", "V", bar_kv)
         for it in range(n_it):
             s, n = it & 1, it >> 1
-            if n > 0:
+            if compute_drain:
+                if it >= 2:
+                    yield from free_stage(it - 2)
+            elif n > 0:
                 yield lambda s=s, n=n: qdo_empty[s].ready(n - 1)
             for nm in ("Q", "dO", "L", "Dv"):
                 M.load((nm, s), (nm, it), qdo_full[s])
+        if compute_drain:
+            if not no_dq or skip == "tail_waits":  # no dQ: the epilogue itself waits for the last dK
+                for t in range(max(n_it - 2, 0), n_it):
+                    yield from free_stage(t)
+            drained.arrive()
 
     def issuer():
         def stage_ready(it):
@@ -161,6 +188,14 @@ def bwd_model(n_it: int, d: int, seed: int, dropout: bool = False, skip: str = "
             M.read(("Dv", s), ("Dv", it))
             M.write(("dS", w, q), ("dS", it))
             ds_full.arrive()
+            if compute_drain and not no_dq:
+                s = it & 1
+                if skip != "drain_wait":
+                    yield lambda it=it: dkq_done.ready(it)
+                M.read((dq_cols, w, q), ("dQ", it))
+                dq_empty.arrive()
+                M.write(("Q" if w == 0 else "dO", s), ("dQ staged", it))
+                staged[s].arrive()
         yield lambda: dkq_done.ready(n_it - 1) and drained.ready(0)
         M.read("dV", n_it)
         M.read("dK", n_it)
@@ -173,14 +208,6 @@ def bwd_model(n_it: int, d: int, seed: int, dropout: bool = False, skip: str = "
             M.read(("dO", 0), "dK staged")
 
     def drain(q):
-        if no_dq:  # the leader only hands each stage back once its MMAs completed
-            if q == 0:
-                for it in range(n_it):
-                    yield lambda it=it: dkq_done.ready(it)
-                    qdo_empty[it & 1].arrive()
-                    if it == n_it - 1:
-                        drained.arrive()
-            return
         for it in range(n_it):
             s = it & 1
             yield lambda it=it: dkq_done.ready(it)
@@ -201,7 +228,9 @@ def bwd_model(n_it: int, d: int, seed: int, dropout: bool = False, skip: str = "
                 if it == n_it - 1:
                     drained.arrive()
 
-    roles = [producer(), issuer()] + [compute(w, q) for w in HALVES for q in QUARTERS] + [drain(q) for q in QUARTERS]
+    roles = [producer(), issuer()] + [compute(w, q) for w in HALVES for q in QUARTERS]
+    if not compute_drain:
+        roles += [drain(q) for q in QUARTERS]
     M.run(roles)
     assert epi.done == 1
 
@@ -222,11 +251,40 @@ def test_no_dq_pipeline_under_random_interleavings(n_it, d):
         bwd_model(n_it, d, seed, no_dq=True)
 
 
+def test_no_dq_tail_waits_would_alias():
+    """Why the producer does not wait for dK(n-2) and dK(n-1) at the end without
+    dQ: nothing holds dK(n-1) back until that thread has seen dK(n-2), so a slow
+    producer's parity wait can fall two phases behind (the model catches it
+    through its slow-role scheduling)."""
+    failures = 0
+    for seed in range(200):
+        try:
+            bwd_model(5, 128, seed, no_dq=True, skip="tail_waits")
+        except AssertionError as e:
+            assert "waiting for phase" in str(e)
+            failures += 1
+    assert failures > 0
+
+
 def test_no_dq_model_detects_a_missing_wait():
     failures = 0
     for seed in range(40):
         try:
             bwd_model(4, 128, seed, no_dq=True, skip="ds_wait")
+        except AssertionError:
+            failures += 1
+    assert failures > 0
+
+
+@pytest.mark.parametrize("skip", ["staged_wait", "drain_wait"])
+def test_compute_drain_model_detects_a_missing_wait(skip):
+    """Not vacuous for the compute-drain layout: a producer that reduce-adds and
+    reloads a stage without waiting for every warp's staged dQ, or compute warps
+    that read dQ before dK / dQ completed, fail the model."""
+    failures = 0
+    for seed in range(40):
+        try:
+            bwd_model(4, 128, seed, skip=skip)
         except AssertionError:
             failures += 1
     assert failures > 0
