@@ -229,22 +229,20 @@ int device_state(DeviceState **out, int *dev_out) {
 }
 
 template <int D, bool CAUSAL, bool DROPOUT, bool FP8 = false>
-cudaError_t launch_fwd(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v, const CUtensorMap &o,
-                       const CUtensorMap &olo, const fa::FwdParams &p, cudaStream_t stream) {
+cudaError_t launch_fwd(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v, const fa::FwdParams &p,
+                       cudaStream_t stream) {
   const dim3 grid(static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.n_qpairs));
   fa::fa_fwd_kernel<D, CAUSAL, DROPOUT, FP8>
-      <<<grid, fa::FwdCfg<D, FP8>::kThreads, fa::FwdCfg<D, FP8>::kSmemBytes, stream>>>(q, k, v, o, olo, p);
+      <<<grid, fa::FwdCfg<D, FP8>::kThreads, fa::FwdCfg<D, FP8>::kSmemBytes, stream>>>(q, k, v, p);
   return cudaGetLastError();
 }
 
 template <bool DROPOUT>
 cudaError_t launch_fwd_any(int d, int causal, const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
-                           const CUtensorMap &o, const CUtensorMap &olo, const fa::FwdParams &p, cudaStream_t s) {
+                           const fa::FwdParams &p, cudaStream_t s) {
   if (d == 64)
-    return causal ? launch_fwd<64, true, DROPOUT>(q, k, v, o, olo, p, s)
-                  : launch_fwd<64, false, DROPOUT>(q, k, v, o, olo, p, s);
-  return causal ? launch_fwd<128, true, DROPOUT>(q, k, v, o, olo, p, s)
-                : launch_fwd<128, false, DROPOUT>(q, k, v, o, olo, p, s);
+    return causal ? launch_fwd<64, true, DROPOUT>(q, k, v, p, s) : launch_fwd<64, false, DROPOUT>(q, k, v, p, s);
+  return causal ? launch_fwd<128, true, DROPOUT>(q, k, v, p, s) : launch_fwd<128, false, DROPOUT>(q, k, v, p, s);
 }
 
 // Dropout mask writer: one thread per (head, query row, 8-key block).
@@ -302,11 +300,11 @@ static int fwd_common(const void *q, const void *k, const void *v, void *o, void
   if (st != FA_OK) return st;
 
   const int BH = B * H;
-  CUtensorMap tq, tk, tv, to, tolo;
-  if (encode_bf16(&tq, q, d, N, BH) || encode_bf16(&tk, k, d, N, BH) || encode_bf16(&tv, v, d, N, BH) ||
-      encode_bf16(&to, o, d, N, BH) || encode_bf16(&tolo, o_lo ? o_lo : o, d, N, BH))
+  CUtensorMap tq, tk, tv;
+  if (encode_bf16(&tq, q, d, N, BH) || encode_bf16(&tk, k, d, N, BH) || encode_bf16(&tv, v, d, N, BH))
     return FA_ERR_CUDA;
   fa::FwdParams p;
+  p.o = static_cast<uint16_t *>(o);
   p.lse = lse;
   p.o_lo = static_cast<uint16_t *>(o_lo);
   p.status = ds->status;
@@ -318,8 +316,8 @@ static int fwd_common(const void *q, const void *k, const void *v, void *o, void
   p.drop = drop ? *drop : fa::DropoutParams{0u, 0u, 0u, 0u, 1.f};
   p.descale_q = p.descale_k = p.descale_v = nullptr;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const cudaError_t e = drop ? launch_fwd_any<true>(d, causal, tq, tk, tv, to, tolo, p, s)
-                             : launch_fwd_any<false>(d, causal, tq, tk, tv, to, tolo, p, s);
+  const cudaError_t e =
+      drop ? launch_fwd_any<true>(d, causal, tq, tk, tv, p, s) : launch_fwd_any<false>(d, causal, tq, tk, tv, p, s);
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -339,11 +337,11 @@ static int fwd_fp8_common(const void *q8, const void *k8, const void *v8, const 
   st = device_state(&ds, nullptr);
   if (st != FA_OK) return st;
   const int BH = B * H;
-  CUtensorMap tq, tk, tv, to;
-  if (encode_u8(&tq, q8, d, N, BH) || encode_u8(&tk, k8, d, N, BH) || encode_u8(&tv, v8, d, N, BH) ||
-      encode_bf16(&to, o, d, N, BH))
+  CUtensorMap tq, tk, tv;
+  if (encode_u8(&tq, q8, d, N, BH) || encode_u8(&tk, k8, d, N, BH) || encode_u8(&tv, v8, d, N, BH))
     return FA_ERR_CUDA;
   fa::FwdParams p;
+  p.o = static_cast<uint16_t *>(o);
   p.lse = lse;
   p.o_lo = nullptr;
   p.status = ds->status;
@@ -357,8 +355,8 @@ static int fwd_fp8_common(const void *q8, const void *k8, const void *v8, const 
   p.descale_k = dk;
   p.descale_v = dv;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const cudaError_t e = causal ? launch_fwd<128, true, false, true>(tq, tk, tv, to, to, p, s)
-                               : launch_fwd<128, false, false, true>(tq, tk, tv, to, to, p, s);
+  const cudaError_t e = causal ? launch_fwd<128, true, false, true>(tq, tk, tv, p, s)
+                               : launch_fwd<128, false, false, true>(tq, tk, tv, p, s);
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -49,6 +49,7 @@
 namespace fa {
 
 struct FwdParams {
+  uint16_t *o;       // [BH, N, D] bf16
   float *lse;        // [BH, N] fp32 (natural log)
   uint16_t *o_lo;    // optional [BH, N, D] bf16: bf16(O_fp32 - O), or nullptr
   int *status;       // device status block
@@ -69,22 +70,21 @@ struct FwdCfg {
   static_assert(!FP8 || D == 128, "the e4m3 forward takes d = 128 (one 128-byte swizzle row per tile row)");
   static constexpr int kElemBytes = FP8 ? 1 : 2;
   static constexpr int kTileBytes = 128 * D * kElemBytes;  // one 128 x D input tile
-  static constexpr int kOutTileBytes = 128 * D * 2;        // one 128 x D bf16 output tile
   static constexpr int kBoxCols = 128 / kElemBytes;        // input elements per 128-byte TMA box row
   static constexpr int kBoxes = kTileBytes / 16384;        // 128-row TMA boxes (16 KB) per input tile
-  static constexpr int kOutBoxes = D / 64;                 // 64-column bf16 boxes per output tile
   static constexpr int kStages = (FP8 || D == 64) ? 8 : 4;  // K/V ring depth
-  // The epilogue stages O and o_lo of both query tiles in the idle ring.
-  static_assert(kStages * kTileBytes >= 4 * kOutTileBytes, "epilogue staging");
+  // The epilogue stages each softmax warp's 32 rows of O and o_lo (bf16, D/2
+  // columns each) in the idle ring.
+  static_assert(kStages * kTileBytes >= 8 * 2 * 32 * D, "epilogue staging");
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kXOff = kKVOff + kStages * kTileBytes;  // half-row maxima [2 tiles][2 halves][128]
   static constexpr int kLOff = kXOff + 2048;                   // half-row sums [2 tiles][2 halves][2][128]
   static constexpr int kBarOff = kLOff + 4096;
-  // mbarriers: q[2], kv_full/kv_empty[kStages], s_full/p_full/pv_done/epi/
-  // drain [2] each (one per query tile), the max and sum exchanges [2][4] (one
-  // per tile and warp pair), two spare; then the TMEM address slot and the abort flag.
-  static constexpr int kNumBars = 2 + 2 * kStages + 26;
+  // mbarriers: q[2], kv_full/kv_empty[kStages], s_full/p_full/pv_done/drain
+  // [2] each (one per query tile), the max and sum exchanges [2][4] (one per
+  // tile and warp pair); then the TMEM address slot and the abort flag.
+  static constexpr int kNumBars = 2 + 2 * kStages + 24;
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kThreads = 352;
   static constexpr int kSoftmaxThreads = 256;
@@ -110,17 +110,32 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
+// Epilogue staging of one warp's 32 rows x D/2 bf16 columns (rows of D bytes):
+// 16-byte chunk c of row r sits at chunk c ^ f(r), with f chosen so that eight
+// rows writing the same chunk, and the chunk-wise read-back, hit distinct banks.
+template <int D>
+__device__ __forceinline__ uint32_t epi_offset(int row, int chunk) {
+  const int f = (D == 128) ? (row & 7) : ((row >> 1) & 3);
+  return static_cast<uint32_t>(row * D + ((chunk ^ f) << 4));
+}
+
+__device__ __forceinline__ uint4 ld_shared_u4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
 // FP8: e4m3 Q, K, V with per-head descale factors (kind::f8f6f4 MMAs, K = 32
 // per instruction); P is rounded to e4m3 for the PV product, four per TMEM
 // column, and O is divided by the fp32 row sum of the unrounded P.
 template <int D, bool CAUSAL, bool DROPOUT = false, bool FP8 = false>
 __global__ void __launch_bounds__(352, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                  const __grid_constant__ CUtensorMap tmOlo, const FwdParams p) {
+                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   static_assert(!(FP8 && DROPOUT), "no dropout in the e4m3 forward");
   using C = FwdCfg<D, FP8>;
   extern __shared__ __align__(1024) uint8_t smem[];
+  if (threadIdx.x == 0) FA_TRACE(1);
 
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
   uint64_t *bar_q = bars + 0;                        // [2]
@@ -129,11 +144,10 @@ __global__ void __launch_bounds__(352, 1)
   uint64_t *bar_s_full = bars + 2 + 2 * C::kStages;  // [2] S_k in TMEM
   uint64_t *bar_p_full = bar_s_full + 2;             // [2] P_k in TMEM (and O_k rescaled)
   uint64_t *bar_pv_done = bar_p_full + 2;            // [2] PV_k completed
-  uint64_t *bar_epi = bar_pv_done + 2;               // [2]
-  uint64_t *bar_drain = bar_epi + 2;                 // [2]
+  uint64_t *bar_drain = bar_pv_done + 2;             // [2] abort path: the issuer's MMAs completed
   uint64_t *bar_x = bar_drain + 2;                   // [2][4] half-row max exchange, per warp pair
   uint64_t *bar_l = bar_x + 8;                       // [2][4] half-row sum exchange, per warp pair
-  static_assert(2 + 2 * C::kStages + 26 == C::kNumBars, "barrier count");
+  static_assert(2 + 2 * C::kStages + 24 == C::kNumBars, "barrier count");
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_l + 8);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -179,7 +193,6 @@ __global__ void __launch_bounds__(352, 1)
       mbar_init(&bar_s_full[k], 1);
       mbar_init(&bar_p_full[k], C::kSoftmaxThreads);
       mbar_init(&bar_pv_done[k], 1);
-      mbar_init(&bar_epi[k], C::kSoftmaxThreads);
       for (int q = 0; q < 4; ++q) {
         // Warps q and q+4 share rows 32q..32q+31 (and an SM sub-partition).
         mbar_init(&bar_x[k * 4 + q], 64);
@@ -209,7 +222,6 @@ __global__ void __launch_bounds__(352, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      tma_prefetch_desc(&tmO);
       mbar_arrive_expect_tx(&bar_q[0], C::kTileBytes);
       for (int b = 0; b < C::kBoxes; ++b)
         tma_load_3d(&tmQ, &bar_q[0], sQ + b * 16384, b * C::kBoxCols, (2 * u) * 128, bh);
@@ -469,11 +481,18 @@ __global__ void __launch_bounds__(352, 1)
     }
     // ---------------------------------------------------------- epilogue
     // Once both tiles' last PV has completed no MMA or load is in flight, so the
-    // K/V ring is free: O_k and its residual are staged there (swizzled) and
-    // written by TMA stores.
+    // K/V ring is free.  Each warp converts its 32 rows x D/2 columns of O_k (and
+    // their rounding residual) to bf16, stages them in its own 2 x 32 x D bytes
+    // of the ring and writes them out with plain coalesced stores: a warp-wide
+    // 16-byte access covers whole D-byte row segments.  Nothing waits for the
+    // stores, so the CTA can exit (and the next CTA start) as soon as they issue.
     ok = ok && __all_sync(0xffffffffu, mbar_wait(ctx, &bar_pv_done[0], (n_k[0] - 1) & 1, kTagPvDone) &&
                                            mbar_wait(ctx, &bar_pv_done[1], (n_k[1] - 1) & 1, kTagPvDone));
     if (ok) tc_fence_after();
+    constexpr int kChunks = D / 16;         // 16-byte chunks in a row's D/2 bf16 columns
+    constexpr int kRowsPerPass = 512 / D;   // rows covered by one warp-wide 16-byte access
+    const uint32_t scr_o = smem_u32(sKV) + warp * (2 * 32 * D);
+    const uint32_t scr_lo = scr_o + 32 * D;
     for (int k = 0; k < 2 && ok; ++k) {
       const int qt = 2 * u + k;
       // Whole-row sums from the two column halves.
@@ -487,67 +506,55 @@ __global__ void __launch_bounds__(352, 1)
       const float lt = l[k] + ls[((h ^ 1) * 2 + 0) * 128 + r];
       const float lrt = lr[k] + ls[((h ^ 1) * 2 + 1) * 128 + r];
       const float inv_l = (FP8 ? p.descale_v[bh] : (DROPOUT ? p.drop.inv_keep : 1.f)) / lrt;
-      const uint32_t st_o = smem_u32(sKV + (2 * k) * C::kOutTileBytes);
-      const uint32_t st_lo = smem_u32(sKV + (2 * k + 1) * C::kOutTileBytes);
-      const uint32_t tO = tmem + lane_off + 256 + k * D;
+      const uint32_t tO = tmem + lane_off + 256 + k * D + h * (D / 2);
+      uint32_t o[D / 2];
 #pragma unroll
-      for (int ch = 0; ch < D / 64; ++ch) {
-        const int col0 = h * (D / 2) + 32 * ch;  // first feature of this 32-column chunk
-        uint32_t o[32];
-        tmem_ld32(tO + col0, o);
-        tmem_wait_ld();
-        uint32_t w[16];
+      for (int ch = 0; ch < D / 64; ++ch) tmem_ld32(tO + 32 * ch, o + 32 * ch);
+      tmem_wait_ld();
+      uint32_t w[D / 4];
 #pragma unroll
-        for (int t = 0; t < 16; ++t)
-          w[t] = pack_bf16(__uint_as_float(o[2 * t]) * inv_l, __uint_as_float(o[2 * t + 1]) * inv_l);
-        const int box = col0 >> 6, chunk0 = (col0 & 63) >> 3;
+      for (int t = 0; t < D / 4; ++t)
+        w[t] = pack_bf16(__uint_as_float(o[2 * t]) * inv_l, __uint_as_float(o[2 * t + 1]) * inv_l);
 #pragma unroll
-        for (int t = 0; t < 4; ++t)
-          st_shared_v4(st_o + box * 16384 + sw128_offset(r, chunk0 + t), w[4 * t], w[4 * t + 1], w[4 * t + 2],
-                       w[4 * t + 3]);
-        if (p.o_lo != nullptr) {
-          // What rounding O to bf16 dropped, itself rounded to bf16: O ~ o + o_lo
-          // to about 16 significant bits (used by the backward's D = rowsum(dO o O)).
+      for (int c = 0; c < kChunks; ++c)
+        st_shared_v4(scr_o + epi_offset<D>(lane, c), w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+      if (p.o_lo != nullptr) {
+        // What rounding O to bf16 dropped, itself rounded to bf16: O ~ o + o_lo
+        // to about 16 significant bits (used by the backward's D = rowsum(dO o O)).
 #pragma unroll
-          for (int t = 0; t < 16; ++t) {
-            const float a = __uint_as_float(o[2 * t]) * inv_l, b = __uint_as_float(o[2 * t + 1]) * inv_l;
-            w[t] = pack_bf16(a - __uint_as_float(w[t] << 16), b - __uint_as_float(w[t] & 0xFFFF0000u));
-          }
+        for (int t = 0; t < D / 4; ++t) {
+          const float a = __uint_as_float(o[2 * t]) * inv_l, b = __uint_as_float(o[2 * t + 1]) * inv_l;
+          w[t] = pack_bf16(a - __uint_as_float(w[t] << 16), b - __uint_as_float(w[t] & 0xFFFF0000u));
+        }
 #pragma unroll
-          for (int t = 0; t < 4; ++t)
-            st_shared_v4(st_lo + box * 16384 + sw128_offset(r, chunk0 + t), w[4 * t], w[4 * t + 1], w[4 * t + 2],
-                         w[4 * t + 3]);
+        for (int c = 0; c < kChunks; ++c)
+          st_shared_v4(scr_lo + epi_offset<D>(lane, c), w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+      }
+      __syncwarp();
+      // Row rq*32 + row of query tile qt; lane reads chunk c of its row.
+      const int c = lane % kChunks;
+      const int row0 = qt * 128 + rq * 32;
+#pragma unroll
+      for (int pass = 0; pass < 32 / kRowsPerPass; ++pass) {
+        const int row = pass * kRowsPerPass + lane / kChunks;
+        if (row0 + row < p.N) {
+          const size_t e = (static_cast<size_t>(bh) * p.N + row0 + row) * D + h * (D / 2) + c * 8;
+          *reinterpret_cast<uint4 *>(p.o + e) = ld_shared_u4(scr_o + epi_offset<D>(row, c));
+          if (p.o_lo != nullptr) *reinterpret_cast<uint4 *>(p.o_lo + e) = ld_shared_u4(scr_lo + epi_offset<D>(row, c));
         }
       }
+      __syncwarp();  // the next tile rewrites this warp's staging
       const int grow = qt * 128 + r;
       if (h == 0 && grow < p.N) p.lse[static_cast<size_t>(bh) * p.N + grow] = (m[k] + log2f(lt)) * 0.69314718055994531f;
     }
-    // Make the generic-proxy smem writes visible to TMA, then one thread stores
-    // both tiles once all softmax threads have written their part.
-    if (ok) {
-      fence_proxy_async_smem();
-      mbar_arrive(&bar_epi[0]);
-      if (warp == 0 && lane == 0 && mbar_wait(ctx, &bar_epi[0], 0, kTagEpi)) {
-        for (int k = 0; k < 2; ++k) {
-          const int qt = 2 * u + k;
-          if (qt * 128 >= p.N) continue;
-          for (int b = 0; b < C::kOutBoxes; ++b) {
-            tma_store_3d(&tmO, sKV + (2 * k) * C::kOutTileBytes + b * 16384, b * 64, qt * 128, bh);
-            if (p.o_lo != nullptr)
-              tma_store_3d(&tmOlo, sKV + (2 * k + 1) * C::kOutTileBytes + b * 16384, b * 64, qt * 128, bh);
-          }
-        }
-        bulk_commit();
-        bulk_wait_read<0>();
-        FA_TRACE(6);
-      }
-    }
+    if (ok && threadIdx.x == 0) FA_TRACE(6);
     __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) FA_TRACE(7);
   if (warp == C::kIssuerWarp) tmem_dealloc(tmem, 512);
 }
 
