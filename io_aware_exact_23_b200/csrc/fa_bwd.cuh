@@ -244,9 +244,7 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
   uint64_t *bar_dq_empty = bars + 11;
   uint64_t *bar_epi = bars + 12;
   uint64_t *bar_drain = bars + 13;
-  uint64_t *bar_drained = bars + 14;   // the dQ drain has finished with every stage buffer
-  uint64_t *bar_stage = bars + 15;     // dQ drain: all 128 rows staged
-  uint64_t *bar_unused = bars + 16;
+  uint64_t *bar_stage = bars + 15;     // dQ drain: all 128 rows staged (bars 14, 16 unused)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -268,7 +266,23 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
 
   const WaitCtx ctx{p.status, abort_flag, kKernelBwd, p.seq};
 
-  if (threadIdx.x == 0) {
+  // Query tile it's Q, dO, LSE*log2(e) and D into stage it % 2.
+  auto load_tile = [&](int it) {
+    const int s = it & 1, i = i0 + it;
+    mbar_arrive_expect_tx(&bar_qdo_full[s], 2 * C::kTile + 1024);
+    for (int b = 0; b < C::kBoxes; ++b) {
+      tma_load_3d(&tmQ, &bar_qdo_full[s], sQ + s * C::kTile + b * 16384, b * 64, i * 128, bh);
+      tma_load_3d(&tmdO, &bar_qdo_full[s], sdO + s * C::kTile + b * 16384, b * 64, i * 128, bh);
+    }
+    const size_t soff = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(i) * 128;
+    bulk_load_1d(sL + s * 128, p.ws_lse2 + soff, 512, &bar_qdo_full[s]);
+    bulk_load_1d(sDv + s * 128, p.ws_D + soff, 512, &bar_qdo_full[s]);
+  };
+
+  // The producer thread sets up the barriers and starts the first loads (K_j, V_j,
+  // the first query tile) before the block-wide barrier, so that they overlap the
+  // TMEM allocation and the other warps' start.
+  if (warp == R::kProducerWarp && lane == 0) {
     *abort_flag = 0;
     if ((smem_u32(smem) & 1023u) != 0) record_failure(ctx, kStatusInternal, 0);
     mbar_init(bar_kv, 1);
@@ -285,11 +299,19 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
     mbar_init(bar_dq_empty, R::kComputeDrain ? 256 : 128);
     mbar_init(bar_epi, 256);
     mbar_init(bar_drain, 1);
-    mbar_init(bar_drained, 1);
     mbar_init(bar_stage, 128);
-    mbar_init(bar_unused, 1);
     fence_barrier_init();
     fence_proxy_async_smem();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmdO);
+    mbar_arrive_expect_tx(bar_kv, 2 * C::kTile);
+    for (int b = 0; b < C::kBoxes; ++b) {
+      tma_load_3d(&tmK, bar_kv, sK + b * 16384, b * 64, j * 128, bh);
+      tma_load_3d(&tmV, bar_kv, sV + b * 16384, b * 64, j * 128, bh);
+    }
+    load_tile(0);
   }
   if (warp == R::kIssuerWarp) {
     tmem_alloc(tmem_slot, 512);
@@ -304,17 +326,8 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
   if (warp == R::kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && !*abort_flag) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      tma_prefetch_desc(&tmdO);
-      mbar_arrive_expect_tx(bar_kv, 2 * C::kTile);
-      for (int b = 0; b < C::kBoxes; ++b) {
-        tma_load_3d(&tmK, bar_kv, sK + b * 16384, b * 64, j * 128, bh);
-        tma_load_3d(&tmV, bar_kv, sV + b * 16384, b * 64, j * 128, bh);
-      }
       bool ok = true;
-      int it = 0;
+      int it = 1;  // K_j, V_j and query tile 0 were loaded before the block-wide barrier
       // Compute-drain layout: query tile t's stage is reloaded (for tile t + 2)
       // once the tile is done with -- after dK(t)'s commit without the dQ
       // product (dK(t+1) is issued behind S^T(t+2), which needs this reload, so
@@ -347,26 +360,15 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
           ok = false;
           break;
         }
-        const int i = i0 + it;
-        mbar_arrive_expect_tx(&bar_qdo_full[s], 2 * C::kTile + 1024);
-        for (int b = 0; b < C::kBoxes; ++b) {
-          tma_load_3d(&tmQ, &bar_qdo_full[s], sQ + s * C::kTile + b * 16384, b * 64, i * 128, bh);
-          tma_load_3d(&tmdO, &bar_qdo_full[s], sdO + s * C::kTile + b * 16384, b * 64, i * 128, bh);
-        }
-        const size_t soff = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(i) * 128;
-        bulk_load_1d(sL + s * 128, p.ws_lse2 + soff, 512, &bar_qdo_full[s]);
-        bulk_load_1d(sDv + s * 128, p.ws_D + soff, 512, &bar_qdo_full[s]);
+        load_tile(it);
       }
-      if constexpr (R::kComputeDrain) {
+      if constexpr (R::kComputeDrain && !NO_DQ) {
         // The last two tiles have no load behind them: reduce-add their staged dQ
-        // here, then let the epilogue have the stage buffers.  Without the dQ
-        // product there is nothing to wait for: the epilogue waits for the last
-        // dK itself, and a wait here for dK(n-2) could miss its phase -- dK(n-1)
-        // does not depend on this thread, so it may complete first.
-        if constexpr (!NO_DQ)
-          for (int t = n_it >= 2 ? n_it - 2 : 0; t < n_it && ok; ++t) ok = free_stage(t);
-        if (ok) mbar_arrive(bar_drained);
-        if constexpr (!NO_DQ) bulk_wait<0>();  // every reduction has landed before the CTA exits
+        // here.  (Without the dQ product there is nothing to wait for, and a wait
+        // here for dK(n-2) could miss its phase: dK(n-1) does not depend on this
+        // thread, so it may complete first.)
+        for (int t = n_it >= 2 ? n_it - 2 : 0; t < n_it && ok; ++t) ok = free_stage(t);
+        bulk_wait<0>();  // every reduction has landed before the CTA exits
       }
       if (!ok) {
         mbar_drain(bar_kv, 0);
@@ -665,14 +667,13 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
       }
     }
     // ---------------------------------------------------------- epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, (n_it - 1) & 1, kBTagDkqDone) &&
-                                             mbar_wait(ctx, bar_drained, 0, kBTagDrained));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, (n_it - 1) & 1, kBTagDkqDone));
     if (ok) {
       tc_fence_after();
-      // Every MMA has completed, every load was consumed and the dQ drain is
-      // done with the stage buffers: stage dV in the Q buffers and dK in the dO
-      // buffers.
-      const uint32_t stV = smem_u32(sQ), stK = smem_u32(sdO);
+      // Every MMA has completed and every load was consumed, so K_j and V_j are
+      // dead: stage dV in V's buffer and dK in K's.  The last tiles' dQ
+      // reduce-adds, still reading the stage buffers, run meanwhile.
+      const uint32_t stV = smem_u32(sV), stK = smem_u32(sK);
       const uint32_t tdK = tmem + lane_off + C::kColdK, tdV = tmem + lane_off + C::kColdV;
 #pragma unroll
       for (int ch = 0; ch < D / 64; ++ch) {
@@ -701,8 +702,8 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
       mbar_arrive(bar_epi);
       if (threadIdx.x == 0 && mbar_wait(ctx, bar_epi, 0, kBTagEpi)) {
         for (int b = 0; b < C::kBoxes; ++b) {
-          tma_store_3d(&tmdV, sQ + b * 16384, b * 64, j * 128, bh);
-          tma_store_3d(&tmdK, sdO + b * 16384, b * 64, j * 128, bh);
+          tma_store_3d(&tmdV, sV + b * 16384, b * 64, j * 128, bh);
+          tma_store_3d(&tmdK, sK + b * 16384, b * 64, j * 128, bh);
         }
         bulk_commit();
         bulk_wait_read<0>();
@@ -764,7 +765,6 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
         // The stage (Q_i, dO_i) is free for the producer: the MMAs that read it
         // completed (bar_dkq_done) and TMA has read the staged dQ.
         mbar_arrive(&bar_qdo_empty[s]);
-        if (it == n_it - 1) mbar_arrive(bar_drained);
       }
       ok = __all_sync(0xffffffffu, ok);
       if (r == 0) FA_TRACE(1024 + it * 2 + 1);

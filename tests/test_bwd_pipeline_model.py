@@ -27,8 +27,8 @@ Roles, as in the kernel (one CTA: key tile j, query tiles it = 0 .. n-1):
   * d = 64 only, four dQ drain warps: read their rows of dQ out of TMEM, stage
     them in tile it's Q / dO stage buffers, and the leader reduce-adds them into
     the accumulator and hands the stage back to the producer;
-  * epilogue: after the last dK / dQ and the drain, dV and dK are staged in the
-    stage-0 buffers and stored.
+  * epilogue: after the last dK / dQ (and, at d = 128, the warp's own drain),
+    dV and dK are staged in V's and K's buffers and stored.
 Checked: no deadlock or phase aliasing; every MMA reads the intended tiles;
 no load lands in a buffer an MMA uses; no role reads a buffer being written or
 writes one an MMA uses; the drain stages each tile's dQ only after the MMAs
@@ -57,7 +57,7 @@ def bwd_model(n_it: int, d: int, seed: int, dropout: bool = False, skip: str = "
     s_full, dp_full = Bar("s_full", 1), Bar("dp_full", 1)
     p_full, ds_full = Bar("p_full", 8), Bar("ds_full", 8)
     dkq_done, dq_empty = Bar("dkq_done", 1), Bar("dq_empty", 8 if compute_drain else 4)
-    epi, drained, stage = Bar("epi", 8), Bar("drained", 1), Bar("stage", 4)
+    epi, stage = Bar("epi", 8), Bar("stage", 4)
     M.tag["dK"] = M.tag["dV"] = 0
     dq_cols = "dPT" if d == 128 else "dQc"  # dQ's TMEM columns
 
@@ -89,7 +89,6 @@ def bwd_model(n_it: int, d: int, seed: int, dropout: bool = False, skip: str = "
             if not no_dq or skip == "tail_waits":  # no dQ: the epilogue itself waits for the last dK
                 for t in range(max(n_it - 2, 0), n_it):
                     yield from free_stage(t)
-            drained.arrive()
 
     def issuer():
         def stage_ready(it):
@@ -196,16 +195,19 @@ def bwd_model(n_it: int, d: int, seed: int, dropout: bool = False, skip: str = "
                 dq_empty.arrive()
                 M.write(("Q" if w == 0 else "dO", s), ("dQ staged", it))
                 staged[s].arrive()
-        yield lambda: dkq_done.ready(n_it - 1) and drained.ready(0)
+        if skip != "epi_wait":
+            yield lambda: dkq_done.ready(n_it - 1)
         M.read("dV", n_it)
         M.read("dK", n_it)
-        M.write(("Q", 0), "dV staged")
-        M.write(("dO", 0), "dK staged")
+        # K_j and V_j are dead once every MMA completed: dV is staged in V's buffer,
+        # dK in K's, while the last dQ reduce-adds may still read the stage buffers
+        M.write("V", "dV staged")
+        M.write("K", "dK staged")
         epi.arrive()
         if w == 0 and q == 0:
             yield lambda: epi.ready(0)
-            M.read(("Q", 0), "dV staged")
-            M.read(("dO", 0), "dK staged")
+            M.read("V", "dV staged")
+            M.read("K", "dK staged")
 
     def drain(q):
         for it in range(n_it):
@@ -225,8 +227,6 @@ def bwd_model(n_it: int, d: int, seed: int, dropout: bool = False, skip: str = "
                 M.read(("Q", s), ("dQ staged", it))
                 M.read(("dO", s), ("dQ staged", it))
                 qdo_empty[s].arrive()
-                if it == n_it - 1:
-                    drained.arrive()
 
     roles = [producer(), issuer()] + [compute(w, q) for w in HALVES for q in QUARTERS]
     if not compute_drain:
@@ -249,6 +249,20 @@ def test_no_dq_pipeline_under_random_interleavings(n_it, d):
     """The deterministic mode's instantiation: no dQ product, no dQ drain."""
     for seed in range(40):
         bwd_model(n_it, d, seed, no_dq=True)
+
+
+@pytest.mark.parametrize("d,no_dq", [(64, False), (128, True), (64, True)])
+def test_epilogue_needs_the_last_dk_dq(d, no_dq):
+    """Not vacuous: an epilogue that stages dK / dV in K's and V's buffers without
+    waiting for the last dK / dQ overwrites operands an MMA still reads.  (At
+    d = 128 with dQ the compute warps' own drain already waits for them.)"""
+    failures = 0
+    for seed in range(40):
+        try:
+            bwd_model(4, d, seed, no_dq=no_dq, skip="epi_wait")
+        except AssertionError:
+            failures += 1
+    assert failures > 0
 
 
 def test_no_dq_tail_waits_would_alias():
