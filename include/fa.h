@@ -75,7 +75,9 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
  * Bytes of scratch fa_bwd needs: an fp32 dQ accumulator [B,H,N,d], plus two
  * fp32 vectors [B,H,Np] with Np = N rounded up to a multiple of 128 -- the
  * per-row D_i = rowsum(dO * O) and LSE_i * log2(e) -- so
- * 4*B*H*(N*d + 2*Np) bytes, rounded up to a multiple of 256.
+ * 4*B*H*(N*d + 2*Np) bytes, rounded up to a multiple of 256; then 256 bytes
+ * more, whose first word counts the work units the backward kernel's CTAs
+ * have taken (one CTA per SM, each taking (head, key tile) units in turn).
  * Returns 0 for unsupported or invalid shapes.
  */
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);

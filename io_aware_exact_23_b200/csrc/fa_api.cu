@@ -393,7 +393,6 @@ static int bwd_common(const void *q, const void *k, const void *v, const void *o
   CUtensorMap maps[7], tdq;
   if (encode_bf16(&maps[0], q, d, N, BH) || encode_bf16(&maps[1], k, d, N, BH) ||
       encode_bf16(&maps[2], v, d, N, BH) || encode_bf16(&maps[3], dO, d, N, BH) ||
-      encode_bf16(&maps[4], dk, d, N, BH) || encode_bf16(&maps[5], dv, d, N, BH) ||
       encode_3d(&maps[6], L.workspace, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, BH, 32) ||
       (deterministic && encode_bf16(&tdq, dq, d, N, BH)))
     return FA_ERR_CUDA;
@@ -623,7 +622,6 @@ extern "C" int fa_bwd_noalloc(const void *q, const void *k, const void *v, const
   CUtensorMap maps[7];
   if (encode_bf16(&maps[0], q, d, N, BH) || encode_bf16(&maps[1], k, d, N, BH) ||
       encode_bf16(&maps[2], v, d, N, BH) || encode_bf16(&maps[3], dO, d, N, BH) ||
-      encode_bf16(&maps[4], dk, d, N, BH) || encode_bf16(&maps[5], dv, d, N, BH) ||
       encode_3d(&maps[6], L.workspace, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, BH, 32))
     return FA_ERR_CUDA;
   cudaError_t e = fa::bwd_launch(L, maps, static_cast<cudaStream_t>(stream));

@@ -57,6 +57,8 @@ struct BwdParams {
   const float *ws_lse2;  // [BH, Npad]  LSE * log2(e), +inf on padded rows
   const float *ws_D;     // [BH, Npad]  rowsum(dO o O), 0 on padded rows
   float *ws_dq;          // [BH, N, D]  fp32 dQ accumulator (zeroed by the preprocess)
+  int *unit_counter;     // units handed out past the first wave (zeroed by the preprocess)
+  uint16_t *dk, *dv;     // [BH, N, D]  bf16 outputs
   int *status;
   int seq;
   int N;
@@ -91,7 +93,8 @@ struct BwdCfg {
   static constexpr int kOffL = kOffdS + 32768;  // [2][128] fp32
   static constexpr int kOffDv = kOffL + 1024;   // [2][128] fp32
   static constexpr int kOffBar = kOffDv + 1024;
-  static constexpr int kNumBars = 17;  // then the TMEM address slot and the abort flag
+  // then the TMEM address slot, the abort flag and the two-slot unit ring
+  static constexpr int kNumBars = 21;
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static constexpr uint32_t kColS = 0, kColdP = 128, kColdK = 256, kColdV = 256 + D;
@@ -115,7 +118,7 @@ struct BwdRoles {
 enum BwdTag : int {
   kBTagKV = 11, kBTagQdoFull = 12, kBTagQdoEmpty = 13, kBTagSFull = 14, kBTagDpFull = 15, kBTagPFull = 16,
   kBTagDsFull = 17, kBTagDvDone = 18, kBTagDkqDone = 19, kBTagDqEmpty = 20, kBTagEpi = 21, kBTagDrained = 22,
-  kBTagStage = 23
+  kBTagStage = 23, kBTagUnit = 24
 };
 
 __device__ __forceinline__ uint32_t bsw128(int row, int chunk) {
@@ -130,7 +133,8 @@ __global__ void __launch_bounds__(256, 4) fa_bwd_pre_kernel(const uint16_t *__re
                                                          const uint16_t *__restrict__ dO,
                                                          const float *__restrict__ lse, float *__restrict__ ws_D,
                                                          float *__restrict__ ws_lse2, float *__restrict__ ws_dq,
-                                                         int N, int Npad, int BH) {
+                                                         int *__restrict__ unit_counter, int N, int Npad, int BH) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) *unit_counter = 0;
   constexpr int LPR = D / 8;     // lanes per row, 16 bytes each
   constexpr int RPW = 32 / LPR;  // rows per warp pass
   constexpr int U = 4;           // passes whose loads are in flight together
@@ -220,33 +224,49 @@ __global__ void __launch_bounds__(256) fa_dq_convert_kernel(const float *__restr
 // query tile (its commit takes the place of dQ(i)'s), the issue order is
 // S^T(0) dP^T(0) | dV(i) S^T(i+1) dK(i) dP^T(i+1) | ... at both head dims, and
 // the producer reloads each Q_i / dO_i stage once dK(i) has completed.
+//
+// Persistent CTAs: the grid holds one CTA per SM (or one per unit, if fewer);
+// CTA c starts on unit c and then takes units from a counter in the workspace,
+// in the same heaviest-first order, each when its current unit is nearly done.  Every per-tile barrier phase and stage
+// runs on t, the CTA's count of query tiles over all its units.  The producer
+// hands each unit to the other roles through a two-slot ring in shared memory,
+// loads the next unit's K_j and V_j once the previous unit's last dK / dQ have
+// completed (after its first query tile), and its stage reloads carry on across
+// units; the next unit's first MMAs overlap the previous unit's last dQ
+// reduce-adds and its epilogue.  A unit's first dV and dK overwrite the
+// accumulators, but they follow P and dS of its first tile, which the compute
+// warps produce only after the previous epilogue has read them.
 template <int D, bool CAUSAL, bool DROPOUT = false, bool NO_DQ = false>
 __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                  const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
                   const __grid_constant__ CUtensorMap tmdQacc, const BwdParams p) {
   using C = BwdCfg<D>;
   using R = BwdRoles<D, NO_DQ>;
   extern __shared__ __align__(1024) uint8_t smem[];
+  if (threadIdx.x == 0) FA_TRACE(1);
 
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
   uint64_t *bar_kv = bars + 0;
   uint64_t *bar_qdo_full = bars + 1;   // [2]
   uint64_t *bar_qdo_empty = bars + 3;  // [2] drain-warp layout: the stage is free again
-  uint64_t *bar_staged = bars + 3;     // [2] compute-drain layout: every compute thread staged its dQ part
+  // [2] compute-drain layout: every compute thread staged its dQ part; without
+  // dQ, the issuer's commit after dK(t).  (A per-stage barrier: a wait on it
+  // cannot fall two phases behind, which one on dkq_done could across units.)
+  uint64_t *bar_staged = bars + 3;
   uint64_t *bar_s_full = bars + 5;
   uint64_t *bar_dp_full = bars + 6;
   uint64_t *bar_p_full = bars + 7;
   uint64_t *bar_ds_full = bars + 8;
-  uint64_t *bar_spare = bars + 9;     // unused
   uint64_t *bar_dkq_done = bars + 10;
   uint64_t *bar_dq_empty = bars + 11;
-  uint64_t *bar_epi = bars + 12;
   uint64_t *bar_drain = bars + 13;
-  uint64_t *bar_stage = bars + 15;     // dQ drain: all 128 rows staged (bars 14, 16 unused)
+  uint64_t *bar_stage = bars + 15;       // dQ drain warps: all 128 rows staged
+  uint64_t *bar_unit_full = bars + 17;   // [2] unit ring: the producer wrote the slot
+  uint64_t *bar_unit_empty = bars + 19;  // [2] unit ring: every consumer warp read it
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  volatile int *unit_ring = reinterpret_cast<volatile int *>(tmem_slot + 2);  // [2]
 
   uint8_t *sK = smem + C::kOffK;
   uint8_t *sV = smem + C::kOffV;
@@ -259,16 +279,14 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int nq = (p.N + 127) / 128;
-  int bh, j;  // head and key tile of this CTA
-  bwd_unit(blockIdx.x, p.BH, nq, bh, j);
-  const int i0 = CAUSAL ? j : 0;
-  const int n_it = nq - i0;
+  const int n_units = p.BH * nq;
+  constexpr int kConsumerWarps = 1 + 8 + (R::kComputeDrain ? 0 : 4);  // issuer, compute, drain
 
   const WaitCtx ctx{p.status, abort_flag, kKernelBwd, p.seq};
 
-  // Query tile it's Q, dO, LSE*log2(e) and D into stage it % 2.
-  auto load_tile = [&](int it) {
-    const int s = it & 1, i = i0 + it;
+  // Query tile i of head bh into stage t % 2: Q, dO, LSE*log2(e), D.
+  auto load_tile = [&](int t, int bh, int i) {
+    const int s = t & 1;
     mbar_arrive_expect_tx(&bar_qdo_full[s], 2 * C::kTile + 1024);
     for (int b = 0; b < C::kBoxes; ++b) {
       tma_load_3d(&tmQ, &bar_qdo_full[s], sQ + s * C::kTile + b * 16384, b * 64, i * 128, bh);
@@ -278,26 +296,35 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
     bulk_load_1d(sL + s * 128, p.ws_lse2 + soff, 512, &bar_qdo_full[s]);
     bulk_load_1d(sDv + s * 128, p.ws_D + soff, 512, &bar_qdo_full[s]);
   };
+  // Key tile j of head bh: K_j, V_j.
+  auto load_kv = [&](int bh, int j) {
+    mbar_arrive_expect_tx(bar_kv, 2 * C::kTile);
+    for (int b = 0; b < C::kBoxes; ++b) {
+      tma_load_3d(&tmK, bar_kv, sK + b * 16384, b * 64, j * 128, bh);
+      tma_load_3d(&tmV, bar_kv, sV + b * 16384, b * 64, j * 128, bh);
+    }
+  };
 
-  // The producer thread sets up the barriers and starts the first loads (K_j, V_j,
-  // the first query tile) before the block-wide barrier, so that they overlap the
-  // TMEM allocation and the other warps' start.
+  // The producer thread sets up the barriers and starts the first unit's loads
+  // (its first query tile, K_j, V_j) before the block-wide barrier, so that they
+  // overlap the TMEM allocation and the other warps' start.
   if (warp == R::kProducerWarp && lane == 0) {
     *abort_flag = 0;
     if ((smem_u32(smem) & 1023u) != 0) record_failure(ctx, kStatusInternal, 0);
     mbar_init(bar_kv, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar_qdo_full[s], 1);
-      mbar_init(&bar_qdo_empty[s], R::kComputeDrain ? 256 : 1);  // bar_staged in that layout
+      // bar_staged in the compute-drain layout: 256 stagers, or the issuer's commit
+      mbar_init(&bar_qdo_empty[s], R::kComputeDrain ? (NO_DQ ? 1 : 256) : 1);
+      mbar_init(&bar_unit_full[s], 1);
+      mbar_init(&bar_unit_empty[s], kConsumerWarps);
     }
     mbar_init(bar_s_full, 1);
     mbar_init(bar_dp_full, 1);
     mbar_init(bar_p_full, 256);
     mbar_init(bar_ds_full, 256);
-    mbar_init(bar_spare, 1);
     mbar_init(bar_dkq_done, 1);
     mbar_init(bar_dq_empty, R::kComputeDrain ? 256 : 128);
-    mbar_init(bar_epi, 256);
     mbar_init(bar_drain, 1);
     mbar_init(bar_stage, 128);
     fence_barrier_init();
@@ -306,12 +333,12 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmdO);
-    mbar_arrive_expect_tx(bar_kv, 2 * C::kTile);
-    for (int b = 0; b < C::kBoxes; ++b) {
-      tma_load_3d(&tmK, bar_kv, sK + b * 16384, b * 64, j * 128, bh);
-      tma_load_3d(&tmV, bar_kv, sV + b * 16384, b * 64, j * 128, bh);
+    if (static_cast<int>(blockIdx.x) < n_units) {
+      int bh, j;
+      bwd_unit(blockIdx.x, p.BH, nq, bh, j);
+      load_tile(0, bh, CAUSAL ? j : 0);
+      load_kv(bh, j);
     }
-    load_tile(0);
   }
   if (warp == R::kIssuerWarp) {
     tmem_alloc(tmem_slot, 512);
@@ -323,59 +350,104 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) FA_TRACE(0);
 
+  // A consumer warp (all lanes) takes unit u from the ring: its index, or -1 (no
+  // more units); take_unit_1 is the same for the issuer's single thread.
+  auto take_unit = [&](int u, int &unit) -> bool {
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_unit_full[u & 1], (u >> 1) & 1, kBTagUnit));
+    if (!ok) return false;
+    unit = unit_ring[u & 1];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bar_unit_empty[u & 1]);
+    return true;
+  };
+  auto take_unit_1 = [&](int u, int &unit) -> bool {
+    if (!mbar_wait(ctx, &bar_unit_full[u & 1], (u >> 1) & 1, kBTagUnit)) return false;
+    unit = unit_ring[u & 1];
+    mbar_arrive(&bar_unit_empty[u & 1]);
+    return true;
+  };
+
   if (warp == R::kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && !*abort_flag) {
       bool ok = true;
-      int it = 1;  // K_j, V_j and query tile 0 were loaded before the block-wide barrier
+      int t = 0;            // query tiles handled so far, over all units
+      int n_loaded = 0;     // query tiles whose loads were issued
+      int n_kv = 0;         // K/V loads issued
+      int stage_row[2] = {0, 0}, stage_bh[2] = {0, 0};  // the tile each stage holds
       // Compute-drain layout: query tile t's stage is reloaded (for tile t + 2)
-      // once the tile is done with -- after dK(t)'s commit without the dQ
-      // product (dK(t+1) is issued behind S^T(t+2), which needs this reload, so
-      // the parity wait cannot fall two phases behind); else once every compute
-      // thread has staged its part of dQ(t) there and this thread has
-      // reduce-added the staged tile into the accumulator (and TMA has read it).
-      auto free_stage = [&](int t) -> bool {
-        const int st = t & 1;
-        if constexpr (NO_DQ) {
-          return mbar_wait(ctx, bar_dkq_done, t & 1, kBTagDkqDone);
-        } else {
-          if (!mbar_wait(ctx, &bar_staged[st], (t >> 1) & 1, kBTagStage)) return false;
+      // once the tile is done with -- after the issuer's commit behind dK(t)
+      // without the dQ product; else once every compute thread has staged its
+      // part of dQ(t) there and this thread has reduce-added the staged tile into
+      // the accumulator (and TMA has read it).
+      auto free_stage = [&](int tt) -> bool {
+        const int st = tt & 1;
+        if (!mbar_wait(ctx, &bar_staged[st], (tt >> 1) & 1, kBTagStage)) return false;
+        if constexpr (!NO_DQ) {
           for (int half = 0; half < 2; ++half)
             for (int b = 0; b < D / 64; ++b)
               tma_reduce_add_3d(&tmdQacc, (half == 0 ? sQ : sdO) + st * C::kTile + b * 16384,
-                                half * (D / 2) + 32 * b, (i0 + t) * 128, bh);
+                                half * (D / 2) + 32 * b, stage_row[st], stage_bh[st]);
           bulk_commit();
           bulk_wait_read<0>();
-          return true;
         }
+        return true;
       };
-      for (; it < n_it; ++it) {
-        const int s = it & 1, n = it >> 1;
-        if constexpr (R::kComputeDrain) {
-          if (it >= 2 && !free_stage(it - 2)) {
-            ok = false;
-            break;
+      int unit = static_cast<int>(blockIdx.x) < n_units ? static_cast<int>(blockIdx.x) : -1;
+      for (int u = 0; ok; ++u) {
+        // Hand unit u (or the end, -1) to the other roles.
+        if (u >= 2 && !(ok = mbar_wait(ctx, &bar_unit_empty[u & 1], ((u >> 1) - 1) & 1, kBTagUnit))) break;
+        unit_ring[u & 1] = unit;
+        mbar_arrive(&bar_unit_full[u & 1]);
+        if (unit < 0) break;
+        int bh, j;
+        bwd_unit(unit, p.BH, nq, bh, j);
+        const int i0 = CAUSAL ? j : 0, n_it = nq - i0;
+        for (int it = 0; it < n_it; ++it) {
+          const int s = t & 1, n = t >> 1;
+          if (u == 0 && it == 0) {  // loaded before the block-wide barrier
+            n_loaded = n_kv = 1;
+          } else {
+            if constexpr (R::kComputeDrain) {
+              if (t >= 2 && !(ok = free_stage(t - 2))) break;
+            } else if (n > 0 && !(ok = mbar_wait(ctx, &bar_qdo_empty[s], (n - 1) & 1, kBTagQdoEmpty))) {
+              break;
+            }
+            load_tile(t, bh, i0 + it);
+            ++n_loaded;
+            if (it == 0) {
+              // K_j, V_j of this unit, once every MMA of the previous one (its last
+              // dK / dQ, committed to bar_dkq_done) has completed.  The wait cannot
+              // fall two phases behind: dK / dQ of tile t need the load below.
+              if (!(ok = mbar_wait(ctx, bar_dkq_done, (t - 1) & 1, kBTagDkqDone))) break;
+              load_kv(bh, j);
+              ++n_kv;
+            }
           }
-        } else if (n > 0 && !mbar_wait(ctx, &bar_qdo_empty[s], (n - 1) & 1, kBTagQdoEmpty)) {
-          ok = false;
-          break;
+          stage_row[s] = (i0 + it) * 128;
+          stage_bh[s] = bh;
+          ++t;
         }
-        load_tile(it);
+        if (!ok) break;
+        // The next unit is claimed once this one's last tile is loaded, a tile or
+        // two before it ends: claimed earlier, it would wait behind this unit while
+        // other CTAs run dry (heaviest-first order needs claims at finish time), and
+        // the atomic's latency still hides behind the remaining tiles.
+        unit = static_cast<int>(gridDim.x) + atomicAdd(p.unit_counter, 1);
+        if (unit >= n_units) unit = -1;
       }
       if constexpr (R::kComputeDrain && !NO_DQ) {
         // The last two tiles have no load behind them: reduce-add their staged dQ
-        // here.  (Without the dQ product there is nothing to wait for, and a wait
-        // here for dK(n-2) could miss its phase: dK(n-1) does not depend on this
-        // thread, so it may complete first.)
-        for (int t = n_it >= 2 ? n_it - 2 : 0; t < n_it && ok; ++t) ok = free_stage(t);
+        // here.  (Without the dQ product there is nothing to wait for.)
+        for (int tt = t >= 2 ? t - 2 : 0; tt < t && ok; ++tt) ok = free_stage(tt);
         bulk_wait<0>();  // every reduction has landed before the CTA exits
       }
-      if (!ok) {
-        mbar_drain(bar_kv, 0);
-        for (int s = 0; s < 2 && s < it; ++s) {
-          const int last = s + ((it - 1 - s) / 2) * 2;
-          mbar_drain(&bar_qdo_full[s], (last >> 1) & 1);
-        }
+      // The last loads have landed before the CTA can exit (immediate unless a
+      // consumer gave up before taking them).
+      if (n_kv > 0) mbar_drain(bar_kv, (n_kv - 1) & 1);
+      for (int s = 0; s < 2 && s < n_loaded; ++s) {
+        const int last = s + ((n_loaded - 1 - s) / 2) * 2;
+        mbar_drain(&bar_qdo_full[s], (last >> 1) & 1);
       }
     }
     __syncwarp();
@@ -393,140 +465,124 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
       const uint64_t dOk0 = make_sdesc(smem_u32(sdO), 16, 1024), dOm0 = make_sdesc(smem_u32(sdO), 16384, 1024);
       const uint32_t tS = tmem + C::kColS, tdP = tmem + C::kColdP, tdK = tmem + C::kColdK;
       const uint32_t tdV = tmem + C::kColdV, tdQ = tmem + C::kColdQ;
-      auto issue_sT = [&](int it) {  // S^T = K_j Q_i^T
-        const uint64_t dQk = sdesc_add(dQk0, (it & 1) * C::kTile);
+      // t: the tile's index over all units (its stage is t % 2); acc: accumulate
+      // into dK / dV (false for a unit's first query tile).
+      auto issue_sT = [&](int t) {  // S^T = K_j Q_i^T
+        const uint64_t dQk = sdesc_add(dQk0, (t & 1) * C::kTile);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
           mma_ss(tS, sdesc_add(dKk, off), sdesc_add(dQk, off), id_ss, ks > 0);
         }
         mma_commit(bar_s_full);
-        FA_TRACE(16 + it * 8 + 0);
+        FA_TRACE(16 + t * 8 + 0);
       };
-      auto issue_dPT = [&](int it) {  // dP^T = V_j dO_i^T
-        const uint64_t dOk = sdesc_add(dOk0, (it & 1) * C::kTile);
+      auto issue_dPT = [&](int t) {  // dP^T = V_j dO_i^T
+        const uint64_t dOk = sdesc_add(dOk0, (t & 1) * C::kTile);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
           mma_ss(tdP, sdesc_add(dVk, off), sdesc_add(dOk, off), id_ss, ks > 0);
         }
         mma_commit(bar_dp_full);
-        FA_TRACE(16 + it * 8 + 1);
+        FA_TRACE(16 + t * 8 + 1);
       };
-      auto issue_dV = [&](int it) {  // dV += P^T dO_i; P^T of query columns 64w.. at S^T columns 64w..64w+31
-        const uint64_t dOm = sdesc_add(dOm0, (it & 1) * C::kTile);
+      auto issue_dV = [&](int t, bool acc) {  // dV += P^T dO_i; P^T of query columns 64w.. at S^T columns 64w..64w+31
+        const uint64_t dOm = sdesc_add(dOm0, (t & 1) * C::kTile);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           mma_ts(tdV, tS + ks * 8 + (ks >= 4 ? 32 : 0), sdesc_add(dOm, ks * 2048), id_kxmn,
-                 (it > 0 || ks > 0) ? 1u : 0u);
-        FA_TRACE(16 + it * 8 + 2);
+                 (acc || ks > 0) ? 1u : 0u);
+        FA_TRACE(16 + t * 8 + 2);
       };
-      auto issue_dK = [&](int it) {  // dK += dS^T Q_i
-        const uint64_t dQm = sdesc_add(dQm0, (it & 1) * C::kTile);
+      auto issue_dK = [&](int t, bool acc) {  // dK += dS^T Q_i
+        const uint64_t dQm = sdesc_add(dQm0, (t & 1) * C::kTile);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_ss(tdK, sdesc_add(dSk, off), sdesc_add(dQm, ks * 2048), id_kxmn, (it > 0 || ks > 0) ? 1u : 0u);
+          mma_ss(tdK, sdesc_add(dSk, off), sdesc_add(dQm, ks * 2048), id_kxmn, (acc || ks > 0) ? 1u : 0u);
         }
       };
-      auto issue_dQ = [&](int it) {  // dQ_i = dS K_j; the dQ drain releases the Q/dO stage after staging through it
+      auto issue_dQ = [&](int t) {  // dQ_i = dS K_j; the dQ drain releases the Q/dO stage after staging through it
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           mma_ss(tdQ, sdesc_add(dSm, ks * 2048), sdesc_add(dKm, ks * 2048), id_mnmn, ks > 0);
         mma_commit(bar_dkq_done);
-        FA_TRACE(16 + it * 8 + 3);
+        FA_TRACE(16 + t * 8 + 3);
       };
-      auto wait_stage = [&](int it) {
-        return mbar_wait(ctx, &bar_qdo_full[it & 1], (it >> 1) & 1, kBTagQdoFull);
+      auto wait_stage = [&](int t) {
+        return mbar_wait(ctx, &bar_qdo_full[t & 1], (t >> 1) & 1, kBTagQdoFull);
       };
       // S^T(i+1) overwrites P^T(i), which dV(i) reads, and dP^T(i+1) the dP^T(i)
       // the compute warps have turned into dS(i): neither waits for an MMA to
       // complete, since one thread issues them all and the pipe runs them in order.
-      bool ok = mbar_wait(ctx, bar_kv, 0, kBTagKV);
-      if (NO_DQ) {
-        // S^T(0) dP^T(0) | dV(i) S^T(i+1) dK(i) dP^T(i+1) | ...: no dQ in TMEM, so
-        // nothing waits for a drain; dK(i)'s commit closes the tile.
-        ok = ok && wait_stage(0);
-        if (ok) {
+      bool ok = true;
+      int t = 0;  // query tiles issued so far, over all units
+      for (int u = 0; ok; ++u) {
+        int unit;
+        if (!(ok = take_unit_1(u, unit))) break;
+        if (unit < 0) break;
+        int bh, j;
+        bwd_unit(unit, p.BH, nq, bh, j);
+        const int n_it = nq - (CAUSAL ? j : 0), t0 = t;
+        if (!(ok = mbar_wait(ctx, bar_kv, u & 1, kBTagKV))) break;
+        if (NO_DQ || D == 64) {
+          // Order S^T(0) dP^T(0) | dV(i) S^T(i+1) dK(i) [dQ(i)] dP^T(i+1) | ...: the
+          // next tile's S^T goes in ahead of dK(i) (and dQ(i), which has columns of
+          // its own at d = 64), so the compute warps start tile i+1 while those run.
+          // Without dQ, dK(i)'s commit closes the tile and frees its stage.
+          if (!(ok = wait_stage(t0))) break;
           tc_fence_after();
-          issue_sT(0);
-          issue_dPT(0);
-        }
-        for (int it = 0; it < n_it && ok; ++it) {
-          ok = mbar_wait(ctx, bar_p_full, it & 1, kBTagPFull);
-          if (!ok) break;
-          tc_fence_after();
-          issue_dV(it);
-          if (it + 1 < n_it) {
-            ok = wait_stage(it + 1);
-            if (!ok) break;
+          issue_sT(t0);
+          issue_dPT(t0);
+          for (int it = 0; it < n_it && ok; ++it) {
+            t = t0 + it;
+            if (!(ok = mbar_wait(ctx, bar_p_full, t & 1, kBTagPFull))) break;
             tc_fence_after();
-            issue_sT(it + 1);
-          }
-          ok = mbar_wait(ctx, bar_ds_full, it & 1, kBTagDsFull);
-          if (!ok) break;
-          tc_fence_after();
-          issue_dK(it);
-          mma_commit(bar_dkq_done);
-          if (it + 1 < n_it) issue_dPT(it + 1);
-        }
-      } else if (D == 128) {
-        // Order S^T(i) dP^T(i) dV(i) dK(i) dQ(i).  dQ(i) accumulates in dP^T's
-        // columns, so dP^T(i+1) also waits for the drain to have read dQ(i).
-        for (int it = 0; it < n_it && ok; ++it) {
-          ok = wait_stage(it);
-          if (!ok) break;
-          tc_fence_after();
-          issue_sT(it);
-          if (it > 0) {
-            ok = mbar_wait(ctx, bar_dq_empty, (it - 1) & 1, kBTagDqEmpty);
-            if (!ok) break;
+            issue_dV(t, it > 0);
+            if (it + 1 < n_it) {
+              if (!(ok = wait_stage(t + 1))) break;
+              tc_fence_after();
+              issue_sT(t + 1);
+            }
+            if (!(ok = mbar_wait(ctx, bar_ds_full, t & 1, kBTagDsFull))) break;
             tc_fence_after();
+            issue_dK(t, it > 0);
+            if constexpr (NO_DQ) {
+              mma_commit(bar_dkq_done);
+              mma_commit(&bar_staged[t & 1]);
+            } else {
+              if (t > 0) {  // dQ of the previous tile has left its columns
+                if (!(ok = mbar_wait(ctx, bar_dq_empty, (t - 1) & 1, kBTagDqEmpty))) break;
+                tc_fence_after();
+              }
+              issue_dQ(t);
+            }
+            if (it + 1 < n_it) issue_dPT(t + 1);
           }
-          issue_dPT(it);
-          ok = mbar_wait(ctx, bar_p_full, it & 1, kBTagPFull);
-          if (!ok) break;
-          tc_fence_after();
-          issue_dV(it);
-          ok = mbar_wait(ctx, bar_ds_full, it & 1, kBTagDsFull);
-          if (!ok) break;
-          tc_fence_after();
-          issue_dK(it);
-          issue_dQ(it);
-        }
-      } else {
-        // Order S^T(0) dP^T(0) | dV(i) S^T(i+1) dK(i) dQ(i) dP^T(i+1) | ...: the
-        // next tile's S^T goes in ahead of dK(i) / dQ(i) (dQ has columns of its
-        // own), so the compute warps start tile i+1 while those run.
-        ok = ok && wait_stage(0);
-        if (ok) {
-          tc_fence_after();
-          issue_sT(0);
-          issue_dPT(0);
-        }
-        for (int it = 0; it < n_it && ok; ++it) {
-          ok = mbar_wait(ctx, bar_p_full, it & 1, kBTagPFull);
-          if (!ok) break;
-          tc_fence_after();
-          issue_dV(it);
-          if (it + 1 < n_it) {
-            ok = wait_stage(it + 1);
-            if (!ok) break;
+        } else {
+          // Order S^T(i) dP^T(i) dV(i) dK(i) dQ(i).  dQ(i) accumulates in dP^T's
+          // columns, so dP^T(i+1) also waits for the drain to have read dQ(i).
+          for (int it = 0; it < n_it && ok; ++it) {
+            t = t0 + it;
+            if (!(ok = wait_stage(t))) break;
             tc_fence_after();
-            issue_sT(it + 1);
-          }
-          ok = mbar_wait(ctx, bar_ds_full, it & 1, kBTagDsFull);
-          if (!ok) break;
-          tc_fence_after();
-          issue_dK(it);
-          if (it > 0) {  // dQ(i-1) has left its columns
-            ok = mbar_wait(ctx, bar_dq_empty, (it - 1) & 1, kBTagDqEmpty);
-            if (!ok) break;
+            issue_sT(t);
+            if (t > 0) {
+              if (!(ok = mbar_wait(ctx, bar_dq_empty, (t - 1) & 1, kBTagDqEmpty))) break;
+              tc_fence_after();
+            }
+            issue_dPT(t);
+            if (!(ok = mbar_wait(ctx, bar_p_full, t & 1, kBTagPFull))) break;
             tc_fence_after();
+            issue_dV(t, it > 0);
+            if (!(ok = mbar_wait(ctx, bar_ds_full, t & 1, kBTagDsFull))) break;
+            tc_fence_after();
+            issue_dK(t, it > 0);
+            issue_dQ(t);
           }
-          issue_dQ(it);
-          if (it + 1 < n_it) issue_dPT(it + 1);
         }
+        t = t0 + n_it;
       }
       if (!ok) {
         mma_commit(bar_drain);
@@ -542,172 +598,201 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
     const uint32_t tS = tmem + lane_off + C::kColS;
     const uint32_t tdP = tmem + lane_off + C::kColdP;
     const uint32_t dS_addr = smem_u32(sdS) + w * 16384;
+    // This warp's 4 KB of the dS tile (the rows it writes there): the epilogue's
+    // staging for its 32 rows x D/2 columns of dV, then of dK.
+    const uint32_t my_dS = smem_u32(sdS) + w * 16384 + (warp & 3) * 4096;
     const float c = p.scale_log2;
     bool ok = !*abort_flag;
-    for (int it = 0; it < n_it && ok; ++it) {
-      const int s = it & 1, n = it >> 1;
-      const int i = i0 + it;
-      ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_s_full, it & 1, kBTagSFull) &&
-                                       mbar_wait(ctx, &bar_qdo_full[s], n & 1, kBTagQdoFull));
-      if (!ok) break;
-      tc_fence_after();
-      if (threadIdx.x == 0) FA_TRACE(16 + it * 8 + 4);
-      // Dropout: keep bit cc for query i*128 + 64w + cc and this thread's key.
-      // The generator's counter blocks run along keys, so the warp draws the
-      // 64 x 32 block together (eight calls per lane) and transposes it through
-      // its own rows of the dS tile, free once the previous tile's dK / dQ are done.
-      uint64_t keep = ~0ull;
-      if constexpr (DROPOUT) {
-        if (it > 0) ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, (it - 1) & 1, kBTagDkqDone));
-        if (!ok) break;
-        const uint32_t slot = smem_u32(sdS) + w * 16384 + (warp & 3) * 4096;  // [64 queries][32 keys] u16
-        const int b = lane & 3;
-        const uint32_t jblk = static_cast<uint32_t>(j * 128 + (warp & 3) * 32) / 8 + b;
-#pragma unroll 1
-        for (int t = 0; t < 8; ++t) {
-          const int ii = (lane >> 2) + 8 * t;
-          const uint4 wv = dropout_words(p.drop, i * 128 + 64 * w + ii, jblk, bh);
-          st_shared_v4(slot + (ii * 32 + 8 * b) * 2, wv.x, wv.y, wv.z, wv.w);
-        }
-        __syncwarp();
-        const uint16_t *draws = reinterpret_cast<const uint16_t *>(sdS + w * 16384 + (warp & 3) * 4096);
-        keep = 0;
-#pragma unroll
-        for (int ii = 0; ii < 64; ++ii) keep |= static_cast<uint64_t>(draws[ii * 32 + lane] >= p.drop.T) << ii;
-        __syncwarp();
+    int t0 = 0;  // this unit's first tile, counted over all units
+    for (int u = 0; ok; ++u) {
+      int unit;
+      if (!(ok = take_unit(u, unit))) break;
+      if (unit < 0) break;
+      // Only the tile count lives through the tile loop (registers are tight): the
+      // head and key tile are derived again where they are needed.
+      int n_it;
+      {
+        int bh_u, j_u;
+        bwd_unit(unit, p.BH, nq, bh_u, j_u);
+        n_it = nq - (CAUSAL ? j_u : 0);
       }
-      uint32_t sv[64];
-      tmem_ld32(tS + 64 * w, sv);
-      tmem_ld32(tS + 64 * w + 32, sv + 32);
-      tmem_wait_ld();
-      const float *lse2 = sL + s * 128 + 64 * w;
-      float pf[64];
-#pragma unroll
-      for (int cc = 0; cc < 64; ++cc) pf[cc] = ex2(fmaf(__uint_as_float(sv[cc]), c, -lse2[cc]));
-      if (CAUSAL && i == j) {
-        // Diagonal tile: key row r is masked for query columns before it.
-#pragma unroll
-        for (int cc = 0; cc < 64; ++cc)
-          if (64 * w + cc < r) pf[cc] = 0.f;
-      }
-      // Z = keep / (keep probability): dV takes (P o Z)^T, dS the dP o Z.
-      auto zval = [&](int cc) { return DROPOUT ? (((keep >> cc) & 1ull) ? p.drop.inv_keep : 0.f) : 1.f; };
-      uint32_t pk[32];
-#pragma unroll
-      for (int t = 0; t < 32; ++t) pk[t] = pack_bf16(pf[2 * t] * zval(2 * t), pf[2 * t + 1] * zval(2 * t + 1));
-      tmem_st32(tS + 64 * w, pk);  // inside the columns this warp has read
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar_p_full);
-      if (threadIdx.x == 0) FA_TRACE(16 + it * 8 + 5);
-
-      ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dp_full, it & 1, kBTagDpFull));
-      // The previous tile's dK / dQ MMAs read dS from smem: wait until they are done.
-      if (ok && it > 0) ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, (it - 1) & 1, kBTagDkqDone));
-      if (!ok) break;
-      tc_fence_after();
-      if (threadIdx.x == 0) FA_TRACE(16 + it * 8 + 6);
-      const float *Dv = sDv + s * 128 + 64 * w;
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t dp[32];
-        tmem_ld32(tdP + 64 * w + 32 * ch, dp);
-        tmem_wait_ld();
-        uint32_t dsk[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          const int c0 = 32 * ch + 2 * t;
-          float z0 = 1.f, z1 = 1.f;
-          if constexpr (DROPOUT) {
-            z0 = keep_bit_fresh(keep, c0) ? p.drop.inv_keep : 0.f;
-            z1 = keep_bit_fresh(keep, c0 + 1) ? p.drop.inv_keep : 0.f;
-          }
-          const float d0 = pf[c0] * (__uint_as_float(dp[2 * t]) * z0 - Dv[c0]);
-          const float d1 = pf[c0 + 1] * (__uint_as_float(dp[2 * t + 1]) * z1 - Dv[c0 + 1]);
-          dsk[t] = pack_bf16(d0, d1);
-        }
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-          st_shared_v4(dS_addr + bsw128(r, 4 * ch + t), dsk[4 * t], dsk[4 * t + 1], dsk[4 * t + 2], dsk[4 * t + 3]);
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar_ds_full);
-      if (threadIdx.x == 0) FA_TRACE(16 + it * 8 + 7);
-      if constexpr (R::kComputeDrain && !NO_DQ) {
-        // dQ drain: once dK(i) and dQ(i) have completed, read this warp's part of
-        // dQ (its lane quarter's rows, columns 64w..) out of TMEM -- which frees
-        // the columns for dP^T(i+1) -- and stage it, scaled, as fp32 in tile i's
-        // Q (w = 0) or dO (w = 1) stage buffer for the producer's reduce-add.
-        ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, it & 1, kBTagDkqDone));
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int t = t0 + it;
+        const int s = t & 1, n = t >> 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_s_full, t & 1, kBTagSFull) &&
+                                         mbar_wait(ctx, &bar_qdo_full[s], n & 1, kBTagQdoFull));
         if (!ok) break;
         tc_fence_after();
-        if (threadIdx.x == 0) FA_TRACE(1024 + it * 2 + 0);
-        uint32_t v[64];
-        const uint32_t tdQ = tmem + lane_off + C::kColdQ + 64 * w;
-        tmem_ld32(tdQ, v);
-        tmem_ld32(tdQ + 32, v + 32);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar_dq_empty);
-        const uint32_t buf = smem_u32((w == 0 ? sQ : sdO) + s * C::kTile);
-#pragma unroll
-        for (int b = 0; b < 2; ++b)
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const int c0 = 32 * b + 4 * t;
-            st_shared_v4(buf + b * 16384 + bsw128(r, t), __float_as_uint(__uint_as_float(v[c0]) * p.scale),
-                         __float_as_uint(__uint_as_float(v[c0 + 1]) * p.scale),
-                         __float_as_uint(__uint_as_float(v[c0 + 2]) * p.scale),
-                         __float_as_uint(__uint_as_float(v[c0 + 3]) * p.scale));
+        if (threadIdx.x == 0) FA_TRACE(16 + t * 8 + 4);
+        // Dropout: keep bit cc for query i*128 + 64w + cc and this thread's key.
+        // The generator's counter blocks run along keys, so the warp draws the
+        // 64 x 32 block together (eight calls per lane) and transposes it through
+        // its own rows of the dS tile, free once the previous tile's dK / dQ are done.
+        uint64_t keep = ~0ull;
+        if constexpr (DROPOUT) {
+          if (t > 0) ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, (t - 1) & 1, kBTagDkqDone));
+          if (!ok) break;
+          int bh, j;
+          bwd_unit(unit, p.BH, nq, bh, j);
+          const int i = (CAUSAL ? j : 0) + it;
+          const uint32_t slot = smem_u32(sdS) + w * 16384 + (warp & 3) * 4096;  // [64 queries][32 keys] u16
+          const int b = lane & 3;
+          const uint32_t jblk = static_cast<uint32_t>(j * 128 + (warp & 3) * 32) / 8 + b;
+#pragma unroll 1
+          for (int q8 = 0; q8 < 8; ++q8) {
+            const int ii = (lane >> 2) + 8 * q8;
+            const uint4 wv = dropout_words(p.drop, i * 128 + 64 * w + ii, jblk, bh);
+            st_shared_v4(slot + (ii * 32 + 8 * b) * 2, wv.x, wv.y, wv.z, wv.w);
           }
-        fence_proxy_async_smem();
-        mbar_arrive(&bar_staged[s]);
-        if (threadIdx.x == 0) FA_TRACE(1024 + it * 2 + 1);
-      }
-    }
-    // ---------------------------------------------------------- epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, (n_it - 1) & 1, kBTagDkqDone));
-    if (ok) {
-      tc_fence_after();
-      // Every MMA has completed and every load was consumed, so K_j and V_j are
-      // dead: stage dV in V's buffer and dK in K's.  The last tiles' dQ
-      // reduce-adds, still reading the stage buffers, run meanwhile.
-      const uint32_t stV = smem_u32(sV), stK = smem_u32(sK);
-      const uint32_t tdK = tmem + lane_off + C::kColdK, tdV = tmem + lane_off + C::kColdV;
-#pragma unroll
-      for (int ch = 0; ch < D / 64; ++ch) {
-        const int col0 = w * (D / 2) + 32 * ch;  // first feature of this 32-column chunk
-        const int box = col0 / 64, chunk0 = (col0 % 64) / 8;
-        uint32_t a[32], pkv[16];
-        tmem_ld32(tdV + col0, a);
-        tmem_wait_ld();
-#pragma unroll
-        for (int t = 0; t < 16; ++t) pkv[t] = pack_bf16(__uint_as_float(a[2 * t]), __uint_as_float(a[2 * t + 1]));
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-          st_shared_v4(stV + box * 16384 + bsw128(r, chunk0 + t), pkv[4 * t], pkv[4 * t + 1], pkv[4 * t + 2],
-                       pkv[4 * t + 3]);
-        tmem_ld32(tdK + col0, a);
-        tmem_wait_ld();
-#pragma unroll
-        for (int t = 0; t < 16; ++t)
-          pkv[t] = pack_bf16(__uint_as_float(a[2 * t]) * p.scale, __uint_as_float(a[2 * t + 1]) * p.scale);
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-          st_shared_v4(stK + box * 16384 + bsw128(r, chunk0 + t), pkv[4 * t], pkv[4 * t + 1], pkv[4 * t + 2],
-                       pkv[4 * t + 3]);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bar_epi);
-      if (threadIdx.x == 0 && mbar_wait(ctx, bar_epi, 0, kBTagEpi)) {
-        for (int b = 0; b < C::kBoxes; ++b) {
-          tma_store_3d(&tmdV, sV + b * 16384, b * 64, j * 128, bh);
-          tma_store_3d(&tmdK, sK + b * 16384, b * 64, j * 128, bh);
+          __syncwarp();
+          const uint16_t *draws = reinterpret_cast<const uint16_t *>(sdS + w * 16384 + (warp & 3) * 4096);
+          keep = 0;
+  #pragma unroll
+          for (int ii = 0; ii < 64; ++ii) keep |= static_cast<uint64_t>(draws[ii * 32 + lane] >= p.drop.T) << ii;
+          __syncwarp();
         }
-        bulk_commit();
-        bulk_wait_read<0>();
+        uint32_t sv[64];
+        tmem_ld32(tS + 64 * w, sv);
+        tmem_ld32(tS + 64 * w + 32, sv + 32);
+        tmem_wait_ld();
+        const float *lse2 = sL + s * 128 + 64 * w;
+        float pf[64];
+  #pragma unroll
+        for (int cc = 0; cc < 64; ++cc) pf[cc] = ex2(fmaf(__uint_as_float(sv[cc]), c, -lse2[cc]));
+        if (CAUSAL && it == 0) {  // the diagonal tile (i = j)
+          // Diagonal tile: key row r is masked for query columns before it.
+  #pragma unroll
+          for (int cc = 0; cc < 64; ++cc)
+            if (64 * w + cc < r) pf[cc] = 0.f;
+        }
+        // Z = keep / (keep probability): dV takes (P o Z)^T, dS the dP o Z.
+        auto zval = [&](int cc) { return DROPOUT ? (((keep >> cc) & 1ull) ? p.drop.inv_keep : 0.f) : 1.f; };
+        uint32_t pk[32];
+  #pragma unroll
+        for (int t = 0; t < 32; ++t) pk[t] = pack_bf16(pf[2 * t] * zval(2 * t), pf[2 * t + 1] * zval(2 * t + 1));
+        tmem_st32(tS + 64 * w, pk);  // inside the columns this warp has read
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_p_full);
+        if (threadIdx.x == 0) FA_TRACE(16 + t * 8 + 5);
+
+        ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dp_full, t & 1, kBTagDpFull));
+        // The previous tile's dK / dQ MMAs read dS from smem: wait until they are done.
+        if (ok && t > 0) ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, (t - 1) & 1, kBTagDkqDone));
+        if (!ok) break;
+        tc_fence_after();
+        if (threadIdx.x == 0) FA_TRACE(16 + t * 8 + 6);
+        const float *Dv = sDv + s * 128 + 64 * w;
+  #pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t dp[32];
+          tmem_ld32(tdP + 64 * w + 32 * ch, dp);
+          tmem_wait_ld();
+          uint32_t dsk[16];
+  #pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const int c0 = 32 * ch + 2 * t;
+            float z0 = 1.f, z1 = 1.f;
+            if constexpr (DROPOUT) {
+              z0 = keep_bit_fresh(keep, c0) ? p.drop.inv_keep : 0.f;
+              z1 = keep_bit_fresh(keep, c0 + 1) ? p.drop.inv_keep : 0.f;
+            }
+            const float d0 = pf[c0] * (__uint_as_float(dp[2 * t]) * z0 - Dv[c0]);
+            const float d1 = pf[c0 + 1] * (__uint_as_float(dp[2 * t + 1]) * z1 - Dv[c0 + 1]);
+            dsk[t] = pack_bf16(d0, d1);
+          }
+  #pragma unroll
+          for (int t = 0; t < 4; ++t)
+            st_shared_v4(dS_addr + bsw128(r, 4 * ch + t), dsk[4 * t], dsk[4 * t + 1], dsk[4 * t + 2], dsk[4 * t + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar_ds_full);
+        if (threadIdx.x == 0) FA_TRACE(16 + t * 8 + 7);
+        if constexpr (R::kComputeDrain && !NO_DQ) {
+          // dQ drain: once dK(i) and dQ(i) have completed, read this warp's part of
+          // dQ (its lane quarter's rows, columns 64w..) out of TMEM -- which frees
+          // the columns for dP^T(i+1) -- and stage it, scaled, as fp32 in tile i's
+          // Q (w = 0) or dO (w = 1) stage buffer for the producer's reduce-add.
+          ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, t & 1, kBTagDkqDone));
+          if (!ok) break;
+          tc_fence_after();
+          if (threadIdx.x == 0) FA_TRACE(1024 + t * 2 + 0);
+          uint32_t v[64];
+          const uint32_t tdQ = tmem + lane_off + C::kColdQ + 64 * w;
+          tmem_ld32(tdQ, v);
+          tmem_ld32(tdQ + 32, v + 32);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar_dq_empty);
+          const uint32_t buf = smem_u32((w == 0 ? sQ : sdO) + s * C::kTile);
+  #pragma unroll
+          for (int b = 0; b < 2; ++b)
+  #pragma unroll
+            for (int t = 0; t < 8; ++t) {
+              const int c0 = 32 * b + 4 * t;
+              st_shared_v4(buf + b * 16384 + bsw128(r, t), __float_as_uint(__uint_as_float(v[c0]) * p.scale),
+                           __float_as_uint(__uint_as_float(v[c0 + 1]) * p.scale),
+                           __float_as_uint(__uint_as_float(v[c0 + 2]) * p.scale),
+                           __float_as_uint(__uint_as_float(v[c0 + 3]) * p.scale));
+            }
+          fence_proxy_async_smem();
+          mbar_arrive(&bar_staged[s]);
+          if (threadIdx.x == 0) FA_TRACE(1024 + t * 2 + 1);
+        }
       }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      // After the unit's last dK / dQ (this warp's own drain already waited at
+      // d = 128 with dQ), dV and dK are final: read this warp's rows out of TMEM
+      // -- which also frees the accumulators for the next unit's first dV, dK
+      // (they follow that unit's first P and dS, which this warp forms later) --
+      // and write them out through the warp's own part of the dS tile (free: the
+      // MMAs that read it completed).  Stores of whole 128-byte row segments, and
+      // nothing waits for them.
+      const int t_last = t0 + n_it - 1;
+      int bh, j;
+      bwd_unit(unit, p.BH, nq, bh, j);
+      if constexpr (!R::kComputeDrain || NO_DQ)
+        ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, t_last & 1, kBTagDkqDone));
+      if (!ok) break;
+      tc_fence_after();
+      if (threadIdx.x == 0) FA_TRACE(2);
+      constexpr int kChunks = D / 16;        // 16-byte chunks in a row's D/2 bf16 columns
+      constexpr int kRowsPerPass = 512 / D;  // rows one warp-wide 16-byte access covers
+      const int row0 = j * 128 + (warp & 3) * 32;  // this warp's first key row
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {  // dV, then dK (times the softmax scale)
+        const uint32_t tacc = tmem + lane_off + (pass == 0 ? C::kColdV : C::kColdK) + w * (D / 2);
+        uint32_t a[D / 2];
+#pragma unroll
+        for (int ch = 0; ch < D / 64; ++ch) tmem_ld32(tacc + 32 * ch, a + 32 * ch);
+        tmem_wait_ld();
+        if (pass == 1) tc_fence_before();  // both accumulators read: the next unit may overwrite them
+        const float f = pass == 0 ? 1.f : p.scale;
+        uint16_t *out = pass == 0 ? p.dv : p.dk;
+#pragma unroll
+        for (int cq = 0; cq < kChunks; ++cq) {
+          uint32_t wv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            wv[e] = pack_bf16(__uint_as_float(a[8 * cq + 2 * e]) * f, __uint_as_float(a[8 * cq + 2 * e + 1]) * f);
+          st_shared_v4(my_dS + epi_offset<D>(lane, cq), wv[0], wv[1], wv[2], wv[3]);
+        }
+        __syncwarp();
+        const int cq = lane % kChunks;
+#pragma unroll
+        for (int ps = 0; ps < 32 / kRowsPerPass; ++ps) {
+          const int row = ps * kRowsPerPass + lane / kChunks;
+          if (row0 + row < p.N) {
+            const size_t e = (static_cast<size_t>(bh) * p.N + row0 + row) * D + w * (D / 2) + cq * 8;
+            *reinterpret_cast<uint4 *>(out + e) = ld_shared_u4(my_dS + epi_offset<D>(row, cq));
+          }
+        }
+        __syncwarp();  // the staging is rewritten by dK, then by the next unit's dS
+      }
+      if (threadIdx.x == 0) FA_TRACE(3);
+      t0 += n_it;
     }
     __syncwarp();
   } else if constexpr (!R::kComputeDrain) {
@@ -721,53 +806,63 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
     const bool leader = (warp == 8 && lane == 0);
     constexpr int kBoxesPerBuf = D / 64;  // 16 KB boxes per stage buffer
     bool ok = !*abort_flag;
-    for (int it = 0; it < n_it && ok; ++it) {
-      const int s = it & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, it & 1, kBTagDkqDone));
-      if (!ok) break;
-      tc_fence_after();
-      if (r == 0) FA_TRACE(1024 + it * 2 + 0);
+    int t0 = 0;  // this unit's first tile, counted over all units
+    for (int u = 0; ok; ++u) {
+      int unit;
+      if (!(ok = take_unit(u, unit))) break;
+      if (unit < 0) break;
+      int bh, j;
+      bwd_unit(unit, p.BH, nq, bh, j);
+      const int i0 = CAUSAL ? j : 0, n_it = nq - i0;
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int t = t0 + it, s = t & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, t & 1, kBTagDkqDone));
+        if (!ok) break;
+        tc_fence_after();
+        if (r == 0) FA_TRACE(1024 + t * 2 + 0);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        // Columns [half*D/2, (half+1)*D/2) -> the Q (half 0) or dO (half 1) stage buffer.
-        uint32_t v[D / 2];
+        for (int half = 0; half < 2; ++half) {
+          // Columns [half*D/2, (half+1)*D/2) -> the Q (half 0) or dO (half 1) stage buffer.
+          uint32_t v[D / 2];
 #pragma unroll
-        for (int ch = 0; ch < D / 64; ++ch) tmem_ld32(tdQ + half * (D / 2) + 32 * ch, v + 32 * ch);
-        tmem_wait_ld();
-        if (half == 1) {
-          tc_fence_before();
-          mbar_arrive(bar_dq_empty);  // dQ is out of TMEM
-        }
-        const uint32_t buf = smem_u32((half == 0 ? sQ : sdO) + s * C::kTile);
-#pragma unroll
-        for (int b = 0; b < kBoxesPerBuf; ++b)
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const int c0 = 32 * b + 4 * t;
-            st_shared_v4(buf + b * 16384 + bsw128(r, t), __float_as_uint(__uint_as_float(v[c0]) * p.scale),
-                         __float_as_uint(__uint_as_float(v[c0 + 1]) * p.scale),
-                         __float_as_uint(__uint_as_float(v[c0 + 2]) * p.scale),
-                         __float_as_uint(__uint_as_float(v[c0 + 3]) * p.scale));
+          for (int ch = 0; ch < D / 64; ++ch) tmem_ld32(tdQ + half * (D / 2) + 32 * ch, v + 32 * ch);
+          tmem_wait_ld();
+          if (half == 1) {
+            tc_fence_before();
+            mbar_arrive(bar_dq_empty);  // dQ is out of TMEM
           }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bar_stage);
-      if (leader) {
-        ok = mbar_wait(ctx, bar_stage, it & 1, kBTagStage);
-        if (ok) {
-          for (int half = 0; half < 2; ++half)
-            for (int b = 0; b < kBoxesPerBuf; ++b)
-              tma_reduce_add_3d(&tmdQacc, (half == 0 ? sQ : sdO) + s * C::kTile + b * 16384,
-                                half * (D / 2) + 32 * b, (i0 + it) * 128, bh);
-          bulk_commit();
-          bulk_wait_read<0>();
+          const uint32_t buf = smem_u32((half == 0 ? sQ : sdO) + s * C::kTile);
+#pragma unroll
+          for (int b = 0; b < kBoxesPerBuf; ++b)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const int c0 = 32 * b + 4 * q;
+              st_shared_v4(buf + b * 16384 + bsw128(r, q), __float_as_uint(__uint_as_float(v[c0]) * p.scale),
+                           __float_as_uint(__uint_as_float(v[c0 + 1]) * p.scale),
+                           __float_as_uint(__uint_as_float(v[c0 + 2]) * p.scale),
+                           __float_as_uint(__uint_as_float(v[c0 + 3]) * p.scale));
+            }
         }
-        // The stage (Q_i, dO_i) is free for the producer: the MMAs that read it
-        // completed (bar_dkq_done) and TMA has read the staged dQ.
-        mbar_arrive(&bar_qdo_empty[s]);
+        fence_proxy_async_smem();
+        mbar_arrive(bar_stage);
+        if (leader) {
+          ok = mbar_wait(ctx, bar_stage, t & 1, kBTagStage);
+          if (ok) {
+            for (int half = 0; half < 2; ++half)
+              for (int b = 0; b < kBoxesPerBuf; ++b)
+                tma_reduce_add_3d(&tmdQacc, (half == 0 ? sQ : sdO) + s * C::kTile + b * 16384,
+                                  half * (D / 2) + 32 * b, (i0 + it) * 128, bh);
+            bulk_commit();
+            bulk_wait_read<0>();
+          }
+          // The stage (Q_i, dO_i) is free for the producer: the MMAs that read it
+          // completed (bar_dkq_done) and TMA has read the staged dQ.
+          mbar_arrive(&bar_qdo_empty[s]);
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        if (r == 0) FA_TRACE(1024 + t * 2 + 1);
       }
-      ok = __all_sync(0xffffffffu, ok);
-      if (r == 0) FA_TRACE(1024 + it * 2 + 1);
+      t0 += n_it;
     }
     if (leader) bulk_wait<0>();  // every reduction has landed before the CTA exits
     __syncwarp();
@@ -776,18 +871,21 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) FA_TRACE(7);
   if (warp == R::kIssuerWarp) tmem_dealloc(tmem, 512);
 }
 
 // ------------------------------------------------------------ host side
 inline int pad128(int n) { return (n + 127) / 128 * 128; }
 
-inline size_t bwd_workspace_bytes(int BH, int N, int d) {
+// Workspace: the fp32 dQ accumulator, the LSE*log2(e) and D vectors, then 256
+// bytes whose first word counts the units fa_bwd_kernel's CTAs have taken.
+inline size_t bwd_workspace_main_bytes(int BH, int N, int d) {
   const size_t dq = static_cast<size_t>(BH) * N * d * 4;
   const size_t vec = static_cast<size_t>(BH) * pad128(N) * 4;
-  const size_t total = dq + 2 * vec;
-  return (total + 255) / 256 * 256;
+  return (dq + 2 * vec + 255) / 256 * 256;
 }
+inline size_t bwd_workspace_bytes(int BH, int N, int d) { return bwd_workspace_main_bytes(BH, N, d) + 256; }
 
 struct BwdLaunch {
   const void *q, *k, *v, *o, *o_lo, *dO;
@@ -822,11 +920,13 @@ inline cudaError_t bwd_set_attributes() {
   return cudaSuccess;
 }
 
+// Persistent grid: one CTA per SM (one resident CTA fits), or one per unit if fewer.
 template <int D, bool CAUSAL, bool DROPOUT, bool NO_DQ = false>
-inline void bwd_main_launch(const CUtensorMap *m, const BwdParams &p, int nkv, cudaStream_t s) {
-  const dim3 grid(static_cast<unsigned>(p.BH) * static_cast<unsigned>(nkv));
+inline void bwd_main_launch(const CUtensorMap *m, const BwdParams &p, int nkv, int num_sms, cudaStream_t s) {
+  const long units = static_cast<long>(p.BH) * nkv;
+  const dim3 grid(static_cast<unsigned>(units < num_sms ? units : num_sms));
   fa_bwd_kernel<D, CAUSAL, DROPOUT, NO_DQ><<<grid, BwdRoles<D, NO_DQ>::kThreads, BwdCfg<D>::kSmemBytes, s>>>(
-      m[0], m[1], m[2], m[3], m[4], m[5], m[6], p);
+      m[0], m[1], m[2], m[3], m[6], p);
 }
 
 // maps: Q, K, V, dO, dK, dV (bf16, 3-D, 64-feature boxes), dQ accumulator
@@ -836,18 +936,20 @@ inline cudaError_t bwd_launch(const BwdLaunch &L, const CUtensorMap *maps, cudaS
   float *ws_dq = static_cast<float *>(L.workspace);
   float *ws_lse2 = ws_dq + static_cast<size_t>(L.BH) * L.N * L.d;
   float *ws_D = ws_lse2 + static_cast<size_t>(L.BH) * Npad;
+  int *counter = reinterpret_cast<int *>(static_cast<uint8_t *>(L.workspace) +
+                                         bwd_workspace_main_bytes(L.BH, L.N, L.d));
   const int pre_grid = L.num_sms * 8;
   cudaError_t e = cudaSuccess;
   if (L.events && (e = cudaEventRecord(L.events[0], s)) != cudaSuccess) return e;
   if (L.d == 64)
     fa_bwd_pre_kernel<64><<<pre_grid, 256, 0, s>>>(static_cast<const uint16_t *>(L.o),
                                                    static_cast<const uint16_t *>(L.o_lo),
-                                                   static_cast<const uint16_t *>(L.dO), L.lse, ws_D, ws_lse2, ws_dq,
+                                                   static_cast<const uint16_t *>(L.dO), L.lse, ws_D, ws_lse2, ws_dq, counter,
                                                    L.N, Npad, L.BH);
   else
     fa_bwd_pre_kernel<128><<<pre_grid, 256, 0, s>>>(static_cast<const uint16_t *>(L.o),
                                                     static_cast<const uint16_t *>(L.o_lo),
-                                                    static_cast<const uint16_t *>(L.dO), L.lse, ws_D, ws_lse2, ws_dq,
+                                                    static_cast<const uint16_t *>(L.dO), L.lse, ws_D, ws_lse2, ws_dq, counter,
                                                     L.N, Npad, L.BH);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -857,6 +959,9 @@ inline cudaError_t bwd_launch(const BwdLaunch &L, const CUtensorMap *maps, cudaS
   p.ws_lse2 = ws_lse2;
   p.ws_D = ws_D;
   p.ws_dq = ws_dq;
+  p.unit_counter = counter;
+  p.dk = static_cast<uint16_t *>(L.dk);
+  p.dv = static_cast<uint16_t *>(L.dv);
   p.status = L.status;
   p.seq = L.seq;
   p.N = L.N;
@@ -868,17 +973,17 @@ inline cudaError_t bwd_launch(const BwdLaunch &L, const CUtensorMap *maps, cudaS
   if (L.drop) p.drop = *L.drop;
   if (L.drop) {
     if (L.d == 64)
-      L.causal ? bwd_main_launch<64, true, true>(maps, p, nkv, s) : bwd_main_launch<64, false, true>(maps, p, nkv, s);
+      L.causal ? bwd_main_launch<64, true, true>(maps, p, nkv, L.num_sms, s) : bwd_main_launch<64, false, true>(maps, p, nkv, L.num_sms, s);
     else
-      L.causal ? bwd_main_launch<128, true, true>(maps, p, nkv, s)
-               : bwd_main_launch<128, false, true>(maps, p, nkv, s);
+      L.causal ? bwd_main_launch<128, true, true>(maps, p, nkv, L.num_sms, s)
+               : bwd_main_launch<128, false, true>(maps, p, nkv, L.num_sms, s);
   } else {
     if (L.d == 64)
-      L.causal ? bwd_main_launch<64, true, false>(maps, p, nkv, s)
-               : bwd_main_launch<64, false, false>(maps, p, nkv, s);
+      L.causal ? bwd_main_launch<64, true, false>(maps, p, nkv, L.num_sms, s)
+               : bwd_main_launch<64, false, false>(maps, p, nkv, L.num_sms, s);
     else
-      L.causal ? bwd_main_launch<128, true, false>(maps, p, nkv, s)
-               : bwd_main_launch<128, false, false>(maps, p, nkv, s);
+      L.causal ? bwd_main_launch<128, true, false>(maps, p, nkv, L.num_sms, s)
+               : bwd_main_launch<128, false, false>(maps, p, nkv, L.num_sms, s);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

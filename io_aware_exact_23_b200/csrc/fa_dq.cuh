@@ -388,17 +388,19 @@ inline cudaError_t bwd_launch_deterministic(const BwdLaunch &L, const CUtensorMa
   float *ws_dq = static_cast<float *>(L.workspace);
   float *ws_lse2 = ws_dq + static_cast<size_t>(L.BH) * L.N * L.d;
   float *ws_D = ws_lse2 + static_cast<size_t>(L.BH) * Npad;
+  int *counter = reinterpret_cast<int *>(static_cast<uint8_t *>(L.workspace) +
+                                         bwd_workspace_main_bytes(L.BH, L.N, L.d));
   const int pre_grid = L.num_sms * 8;
   // No dQ accumulator here (dQ comes from fa_dq_kernel): nullptr skips its zeroing.
   if (L.d == 64)
     fa_bwd_pre_kernel<64><<<pre_grid, 256, 0, s>>>(static_cast<const uint16_t *>(L.o),
                                                    static_cast<const uint16_t *>(L.o_lo),
-                                                   static_cast<const uint16_t *>(L.dO), L.lse, ws_D, ws_lse2, nullptr,
+                                                   static_cast<const uint16_t *>(L.dO), L.lse, ws_D, ws_lse2, nullptr, counter,
                                                    L.N, Npad, L.BH);
   else
     fa_bwd_pre_kernel<128><<<pre_grid, 256, 0, s>>>(static_cast<const uint16_t *>(L.o),
                                                     static_cast<const uint16_t *>(L.o_lo),
-                                                    static_cast<const uint16_t *>(L.dO), L.lse, ws_D, ws_lse2, nullptr,
+                                                    static_cast<const uint16_t *>(L.dO), L.lse, ws_D, ws_lse2, nullptr, counter,
                                                     L.N, Npad, L.BH);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -407,6 +409,9 @@ inline cudaError_t bwd_launch_deterministic(const BwdLaunch &L, const CUtensorMa
   p.ws_lse2 = ws_lse2;
   p.ws_D = ws_D;
   p.ws_dq = ws_dq;
+  p.unit_counter = counter;
+  p.dk = static_cast<uint16_t *>(L.dk);
+  p.dv = static_cast<uint16_t *>(L.dv);
   p.status = L.status;
   p.seq = L.seq;
   p.N = L.N;
@@ -417,11 +422,11 @@ inline cudaError_t bwd_launch_deterministic(const BwdLaunch &L, const CUtensorMa
   const int nkv = Npad / 128;
   // dK, dV from the fused kernel without its dQ product (NO_DQ).
   if (L.d == 64)
-    L.causal ? bwd_main_launch<64, true, false, true>(maps, p, nkv, s)
-             : bwd_main_launch<64, false, false, true>(maps, p, nkv, s);
+    L.causal ? bwd_main_launch<64, true, false, true>(maps, p, nkv, L.num_sms, s)
+             : bwd_main_launch<64, false, false, true>(maps, p, nkv, L.num_sms, s);
   else
-    L.causal ? bwd_main_launch<128, true, false, true>(maps, p, nkv, s)
-             : bwd_main_launch<128, false, false, true>(maps, p, nkv, s);
+    L.causal ? bwd_main_launch<128, true, false, true>(maps, p, nkv, L.num_sms, s)
+             : bwd_main_launch<128, false, false, true>(maps, p, nkv, L.num_sms, s);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   DqParams q;

@@ -110,20 +110,6 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-// Epilogue staging of one warp's 32 rows x D/2 bf16 columns (rows of D bytes):
-// 16-byte chunk c of row r sits at chunk c ^ f(r), with f chosen so that eight
-// rows writing the same chunk, and the chunk-wise read-back, hit distinct banks.
-template <int D>
-__device__ __forceinline__ uint32_t epi_offset(int row, int chunk) {
-  const int f = (D == 128) ? (row & 7) : ((row >> 1) & 3);
-  return static_cast<uint32_t>(row * D + ((chunk ^ f) << 4));
-}
-
-__device__ __forceinline__ uint4 ld_shared_u4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
 
 // FP8: e4m3 Q, K, V with per-head descale factors (kind::f8f6f4 MMAs, K = 32
 // per instruction); P is rounded to e4m3 for the PV product, four per TMEM

@@ -387,6 +387,22 @@ __device__ __forceinline__ void red_add_v4(float *gptr, float a, float b, float 
                : "memory");
 }
 
+__device__ __forceinline__ uint4 ld_shared_u4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// Epilogue staging of one warp's 32 rows x D/2 bf16 columns (rows of D bytes),
+// for stores of whole row segments: 16-byte chunk c of row r sits at chunk
+// c ^ f(r), with f chosen so that eight rows writing the same chunk, and the
+// chunk-wise read-back, hit distinct banks.
+template <int D>
+__device__ __forceinline__ uint32_t epi_offset(int row, int chunk) {
+  const int f = (D == 128) ? (row & 7) : ((row >> 1) & 3);
+  return static_cast<uint32_t>(row * D + ((chunk ^ f) << 4));
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
