@@ -19,10 +19,15 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kStatusInts = 8;
+// The forward's unit counters: a launch uses slot seq % kFwdCounterSlots, zeroed on
+// its stream just before it, so launches in flight at the same time use distinct
+// slots unless kFwdCounterSlots of them are.
+constexpr int kFwdCounterSlots = 4096;
 
 struct DeviceState {
   bool ready = false;
-  int *status = nullptr;  // kStatusInts ints, device memory
+  int *status = nullptr;        // kStatusInts ints, device memory
+  int *fwd_counters = nullptr;  // kFwdCounterSlots ints, after the status block
   int num_sms = 0;
   bool attrs_set = false;
 };
@@ -190,16 +195,18 @@ int device_state(DeviceState **out, int *dev_out) {
     }
     if (major != 10 || minor != 0) return FA_ERR_UNSUPPORTED;
     int *st = nullptr;
-    if (cudaMalloc(&st, kStatusInts * sizeof(int)) != cudaSuccess) {
+    const size_t bytes = (kStatusInts + kFwdCounterSlots) * sizeof(int);
+    if (cudaMalloc(&st, bytes) != cudaSuccess) {
       cudaGetLastError();
       return FA_ERR_CUDA;
     }
-    if (cudaMemset(st, 0, kStatusInts * sizeof(int)) != cudaSuccess) {
+    if (cudaMemset(st, 0, bytes) != cudaSuccess) {
       cudaGetLastError();
       cudaFree(st);
       return FA_ERR_CUDA;
     }
     s.status = st;
+    s.fwd_counters = st + kStatusInts;
     s.num_sms = sms;
     s.ready = true;
   }
@@ -228,10 +235,12 @@ int device_state(DeviceState **out, int *dev_out) {
   return FA_OK;
 }
 
+// Persistent grid: one CTA per SM (one resident CTA fits), or one per unit if fewer.
 template <int D, bool CAUSAL, bool DROPOUT, bool FP8 = false>
 cudaError_t launch_fwd(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v, const fa::FwdParams &p,
-                       cudaStream_t stream) {
-  const dim3 grid(static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.n_qpairs));
+                       int num_sms, cudaStream_t stream) {
+  const long units = static_cast<long>(p.BH) * p.n_qpairs;
+  const dim3 grid(static_cast<unsigned>(units < num_sms ? units : num_sms));
   fa::fa_fwd_kernel<D, CAUSAL, DROPOUT, FP8>
       <<<grid, fa::FwdCfg<D, FP8>::kThreads, fa::FwdCfg<D, FP8>::kSmemBytes, stream>>>(q, k, v, p);
   return cudaGetLastError();
@@ -239,10 +248,21 @@ cudaError_t launch_fwd(const CUtensorMap &q, const CUtensorMap &k, const CUtenso
 
 template <bool DROPOUT>
 cudaError_t launch_fwd_any(int d, int causal, const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
-                           const fa::FwdParams &p, cudaStream_t s) {
+                           const fa::FwdParams &p, int n, cudaStream_t s) {
   if (d == 64)
-    return causal ? launch_fwd<64, true, DROPOUT>(q, k, v, p, s) : launch_fwd<64, false, DROPOUT>(q, k, v, p, s);
-  return causal ? launch_fwd<128, true, DROPOUT>(q, k, v, p, s) : launch_fwd<128, false, DROPOUT>(q, k, v, p, s);
+    return causal ? launch_fwd<64, true, DROPOUT>(q, k, v, p, n, s) : launch_fwd<64, false, DROPOUT>(q, k, v, p, n, s);
+  return causal ? launch_fwd<128, true, DROPOUT>(q, k, v, p, n, s) : launch_fwd<128, false, DROPOUT>(q, k, v, p, n, s);
+}
+
+// Zero the launch's unit-counter slot on its stream.
+int fwd_counter(DeviceState *ds, int seq, cudaStream_t s, int **out) {
+  int *c = ds->fwd_counters + (seq & (kFwdCounterSlots - 1));
+  if (cudaMemsetAsync(c, 0, sizeof(int), s) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  *out = c;
+  return FA_OK;
 }
 
 // Dropout mask writer: one thread per (head, query row, 8-key block).
@@ -316,8 +336,11 @@ static int fwd_common(const void *q, const void *k, const void *v, void *o, void
   p.drop = drop ? *drop : fa::DropoutParams{0u, 0u, 0u, 0u, 1.f};
   p.descale_q = p.descale_k = p.descale_v = nullptr;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const cudaError_t e =
-      drop ? launch_fwd_any<true>(d, causal, tq, tk, tv, p, s) : launch_fwd_any<false>(d, causal, tq, tk, tv, p, s);
+  st = fwd_counter(ds, p.seq, s, &p.unit_counter);
+  if (st != FA_OK) return st;
+  const int n = ds->num_sms;
+  const cudaError_t e = drop ? launch_fwd_any<true>(d, causal, tq, tk, tv, p, n, s)
+                             : launch_fwd_any<false>(d, causal, tq, tk, tv, p, n, s);
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -355,8 +378,10 @@ static int fwd_fp8_common(const void *q8, const void *k8, const void *v8, const 
   p.descale_k = dk;
   p.descale_v = dv;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const cudaError_t e = causal ? launch_fwd<128, true, false, true>(tq, tk, tv, p, s)
-                               : launch_fwd<128, false, false, true>(tq, tk, tv, p, s);
+  st = fwd_counter(ds, p.seq, s, &p.unit_counter);
+  if (st != FA_OK) return st;
+  const cudaError_t e = causal ? launch_fwd<128, true, false, true>(tq, tk, tv, p, ds->num_sms, s)
+                               : launch_fwd<128, false, false, true>(tq, tk, tv, p, ds->num_sms, s);
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
