@@ -764,21 +764,23 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
 #pragma unroll
       for (int pass = 0; pass < 2; ++pass) {  // dV, then dK (times the softmax scale)
         const uint32_t tacc = tmem + lane_off + (pass == 0 ? C::kColdV : C::kColdK) + w * (D / 2);
-        uint32_t a[D / 2];
-#pragma unroll
-        for (int ch = 0; ch < D / 64; ++ch) tmem_ld32(tacc + 32 * ch, a + 32 * ch);
-        tmem_wait_ld();
-        if (pass == 1) tc_fence_before();  // both accumulators read: the next unit may overwrite them
         const float f = pass == 0 ? 1.f : p.scale;
         uint16_t *out = pass == 0 ? p.dv : p.dk;
 #pragma unroll
-        for (int cq = 0; cq < kChunks; ++cq) {
-          uint32_t wv[4];
+        for (int ch = 0; ch < D / 64; ++ch) {  // 32 columns at a time (registers are tight)
+          uint32_t a[32];
+          tmem_ld32(tacc + 32 * ch, a);
+          tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            wv[e] = pack_bf16(__uint_as_float(a[8 * cq + 2 * e]) * f, __uint_as_float(a[8 * cq + 2 * e + 1]) * f);
-          st_shared_v4(my_dS + epi_offset<D>(lane, cq), wv[0], wv[1], wv[2], wv[3]);
+          for (int cq = 0; cq < 4; ++cq) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              wv[e] = pack_bf16(__uint_as_float(a[8 * cq + 2 * e]) * f, __uint_as_float(a[8 * cq + 2 * e + 1]) * f);
+            st_shared_v4(my_dS + epi_offset<D>(lane, 4 * ch + cq), wv[0], wv[1], wv[2], wv[3]);
+          }
         }
+        if (pass == 1) tc_fence_before();  // both accumulators read: the next unit may overwrite them
         __syncwarp();
         const int cq = lane % kChunks;
 #pragma unroll
