@@ -87,14 +87,18 @@ struct BwdCfg {
   static constexpr int kBoxes = D / 64;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTile;
-  static constexpr int kOffQ = 2 * kTile;   // [2]
-  static constexpr int kOffdO = 4 * kTile;  // [2]
-  static constexpr int kOffdS = 6 * kTile;  // 128 x 128 bf16
-  static constexpr int kOffL = kOffdS + 32768;  // [2][128] fp32
-  static constexpr int kOffDv = kOffL + 1024;   // [2][128] fp32
-  static constexpr int kOffBar = kOffDv + 1024;
+  // Q_i / dO_i stages: three at d = 64, where shared memory has room, so that a
+  // stage's reload (behind the drain of the tile two back) has a tile of slack;
+  // two at d = 128, where shared memory is full.
+  static constexpr int kQStages = (D == 64) ? 3 : 2;
+  static constexpr int kOffQ = 2 * kTile;                 // [kQStages]
+  static constexpr int kOffdO = (2 + kQStages) * kTile;   // [kQStages]
+  static constexpr int kOffdS = (2 + 2 * kQStages) * kTile;  // 128 x 128 bf16
+  static constexpr int kOffL = kOffdS + 32768;                // [kQStages][128] fp32
+  static constexpr int kOffDv = kOffL + 512 * kQStages;       // [kQStages][128] fp32
+  static constexpr int kOffBar = kOffDv + 512 * kQStages;
   // then the TMEM address slot, the abort flag and the two-slot unit ring
-  static constexpr int kNumBars = 21;
+  static constexpr int kNumBars = 2 * kQStages + 14;
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static constexpr uint32_t kColS = 0, kColdP = 128, kColdK = 256, kColdV = 256 + D;
@@ -246,24 +250,27 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem[];
   if (threadIdx.x == 0) FA_TRACE(1);
 
+  constexpr int S = C::kQStages;  // query tile t sits in stage t % S
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
   uint64_t *bar_kv = bars + 0;
-  uint64_t *bar_qdo_full = bars + 1;   // [2]
-  uint64_t *bar_qdo_empty = bars + 3;  // [2] drain-warp layout: the stage is free again
-  // [2] compute-drain layout: every compute thread staged its dQ part; without
+  uint64_t *bar_qdo_full = bars + 1;       // [S]
+  uint64_t *bar_qdo_empty = bars + 1 + S;  // [S] drain-warp layout: the stage is free again
+  // [S] compute-drain layout: every compute thread staged its dQ part; without
   // dQ, the issuer's commit after dK(t).  (A per-stage barrier: a wait on it
   // cannot fall two phases behind, which one on dkq_done could across units.)
-  uint64_t *bar_staged = bars + 3;
-  uint64_t *bar_s_full = bars + 5;
-  uint64_t *bar_dp_full = bars + 6;
-  uint64_t *bar_p_full = bars + 7;
-  uint64_t *bar_ds_full = bars + 8;
-  uint64_t *bar_dkq_done = bars + 10;
-  uint64_t *bar_dq_empty = bars + 11;
-  uint64_t *bar_drain = bars + 13;
-  uint64_t *bar_stage = bars + 15;       // dQ drain warps: all 128 rows staged
-  uint64_t *bar_unit_full = bars + 17;   // [2] unit ring: the producer wrote the slot
-  uint64_t *bar_unit_empty = bars + 19;  // [2] unit ring: every consumer warp read it
+  uint64_t *bar_staged = bar_qdo_empty;
+  uint64_t *bar_s_full = bars + 1 + 2 * S;
+  uint64_t *bar_dp_full = bar_s_full + 1;
+  uint64_t *bar_p_full = bar_s_full + 2;
+  uint64_t *bar_ds_full = bar_s_full + 3;
+  uint64_t *bar_dkq_done = bar_s_full + 4;
+  uint64_t *bar_dq_empty = bar_s_full + 5;
+  uint64_t *bar_drain = bar_s_full + 6;
+  uint64_t *bar_stage = bar_s_full + 7;       // dQ drain warps: all 128 rows staged
+  uint64_t *bar_unit_full = bar_s_full + 8;   // [2] unit ring: the producer wrote the slot
+  uint64_t *bar_unit_empty = bar_s_full + 10; // [2] unit ring: every consumer warp read it
+  uint64_t *bar_kv_free = bar_s_full + 12;    // a unit's last MMA completed: K_j, V_j are dead
+  static_assert(1 + 2 * S + 13 == C::kNumBars, "barrier count");
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   volatile int *unit_ring = reinterpret_cast<volatile int *>(tmem_slot + 2);  // [2]
@@ -284,9 +291,9 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
 
   const WaitCtx ctx{p.status, abort_flag, kKernelBwd, p.seq};
 
-  // Query tile i of head bh into stage t % 2: Q, dO, LSE*log2(e), D.
+  // Query tile i of head bh into stage t % S: Q, dO, LSE*log2(e), D.
   auto load_tile = [&](int t, int bh, int i) {
-    const int s = t & 1;
+    const int s = t % S;
     mbar_arrive_expect_tx(&bar_qdo_full[s], 2 * C::kTile + 1024);
     for (int b = 0; b < C::kBoxes; ++b) {
       tma_load_3d(&tmQ, &bar_qdo_full[s], sQ + s * C::kTile + b * 16384, b * 64, i * 128, bh);
@@ -312,10 +319,12 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
     *abort_flag = 0;
     if ((smem_u32(smem) & 1023u) != 0) record_failure(ctx, kStatusInternal, 0);
     mbar_init(bar_kv, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&bar_qdo_full[s], 1);
       // bar_staged in the compute-drain layout: 256 stagers, or the issuer's commit
       mbar_init(&bar_qdo_empty[s], R::kComputeDrain ? (NO_DQ ? 1 : 256) : 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&bar_unit_full[s], 1);
       mbar_init(&bar_unit_empty[s], kConsumerWarps);
     }
@@ -327,6 +336,7 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
     mbar_init(bar_dq_empty, R::kComputeDrain ? 256 : 128);
     mbar_init(bar_drain, 1);
     mbar_init(bar_stage, 128);
+    mbar_init(bar_kv_free, 1);
     fence_barrier_init();
     fence_proxy_async_smem();
     tma_prefetch_desc(&tmQ);
@@ -374,15 +384,15 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
       int t = 0;            // query tiles handled so far, over all units
       int n_loaded = 0;     // query tiles whose loads were issued
       int n_kv = 0;         // K/V loads issued
-      int stage_row[2] = {0, 0}, stage_bh[2] = {0, 0};  // the tile each stage holds
-      // Compute-drain layout: query tile t's stage is reloaded (for tile t + 2)
+      int stage_row[S] = {}, stage_bh[S] = {};  // the tile each stage holds
+      // Compute-drain layout: query tile t's stage is reloaded (for tile t + S)
       // once the tile is done with -- after the issuer's commit behind dK(t)
       // without the dQ product; else once every compute thread has staged its
       // part of dQ(t) there and this thread has reduce-added the staged tile into
       // the accumulator (and TMA has read it).
       auto free_stage = [&](int tt) -> bool {
-        const int st = tt & 1;
-        if (!mbar_wait(ctx, &bar_staged[st], (tt >> 1) & 1, kBTagStage)) return false;
+        const int st = tt % S;
+        if (!mbar_wait(ctx, &bar_staged[st], (tt / S) & 1, kBTagStage)) return false;
         if constexpr (!NO_DQ) {
           for (int half = 0; half < 2; ++half)
             for (int b = 0; b < D / 64; ++b)
@@ -404,22 +414,23 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
         bwd_unit(unit, p.BH, nq, bh, j);
         const int i0 = CAUSAL ? j : 0, n_it = nq - i0;
         for (int it = 0; it < n_it; ++it) {
-          const int s = t & 1, n = t >> 1;
+          const int s = t % S, n = t / S;
           if (u == 0 && it == 0) {  // loaded before the block-wide barrier
             n_loaded = n_kv = 1;
           } else {
             if constexpr (R::kComputeDrain) {
-              if (t >= 2 && !(ok = free_stage(t - 2))) break;
+              if (t >= S && !(ok = free_stage(t - S))) break;
             } else if (n > 0 && !(ok = mbar_wait(ctx, &bar_qdo_empty[s], (n - 1) & 1, kBTagQdoEmpty))) {
               break;
             }
             load_tile(t, bh, i0 + it);
             ++n_loaded;
             if (it == 0) {
-              // K_j, V_j of this unit, once every MMA of the previous one (its last
-              // dK / dQ, committed to bar_dkq_done) has completed.  The wait cannot
-              // fall two phases behind: dK / dQ of tile t need the load below.
-              if (!(ok = mbar_wait(ctx, bar_dkq_done, (t - 1) & 1, kBTagDkqDone))) break;
+              // K_j, V_j of this unit, once every MMA of the previous one has
+              // completed (the issuer's per-unit commit; a wait on dkq_done could
+              // miss its phase, with three stages this thread runs far enough
+              // ahead).  The wait cannot alias: the next commit needs this load.
+              if (!(ok = mbar_wait(ctx, bar_kv_free, (u - 1) & 1, kBTagKV))) break;
               load_kv(bh, j);
               ++n_kv;
             }
@@ -437,17 +448,17 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
         if (unit >= n_units) unit = -1;
       }
       if constexpr (R::kComputeDrain && !NO_DQ) {
-        // The last two tiles have no load behind them: reduce-add their staged dQ
+        // The last S tiles have no load behind them: reduce-add their staged dQ
         // here.  (Without the dQ product there is nothing to wait for.)
-        for (int tt = t >= 2 ? t - 2 : 0; tt < t && ok; ++tt) ok = free_stage(tt);
+        for (int tt = t >= S ? t - S : 0; tt < t && ok; ++tt) ok = free_stage(tt);
         bulk_wait<0>();  // every reduction has landed before the CTA exits
       }
       // The last loads have landed before the CTA can exit (immediate unless a
       // consumer gave up before taking them).
       if (n_kv > 0) mbar_drain(bar_kv, (n_kv - 1) & 1);
-      for (int s = 0; s < 2 && s < n_loaded; ++s) {
-        const int last = s + ((n_loaded - 1 - s) / 2) * 2;
-        mbar_drain(&bar_qdo_full[s], (last >> 1) & 1);
+      for (int s = 0; s < S && s < n_loaded; ++s) {
+        const int last = s + ((n_loaded - 1 - s) / S) * S;
+        mbar_drain(&bar_qdo_full[s], (last / S) & 1);
       }
     }
     __syncwarp();
@@ -468,7 +479,7 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
       // t: the tile's index over all units (its stage is t % 2); acc: accumulate
       // into dK / dV (false for a unit's first query tile).
       auto issue_sT = [&](int t) {  // S^T = K_j Q_i^T
-        const uint64_t dQk = sdesc_add(dQk0, (t & 1) * C::kTile);
+        const uint64_t dQk = sdesc_add(dQk0, (t % S) * C::kTile);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
@@ -478,7 +489,7 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
         FA_TRACE(16 + t * 8 + 0);
       };
       auto issue_dPT = [&](int t) {  // dP^T = V_j dO_i^T
-        const uint64_t dOk = sdesc_add(dOk0, (t & 1) * C::kTile);
+        const uint64_t dOk = sdesc_add(dOk0, (t % S) * C::kTile);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
@@ -488,7 +499,7 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
         FA_TRACE(16 + t * 8 + 1);
       };
       auto issue_dV = [&](int t, bool acc) {  // dV += P^T dO_i; P^T of query columns 64w.. at S^T columns 64w..64w+31
-        const uint64_t dOm = sdesc_add(dOm0, (t & 1) * C::kTile);
+        const uint64_t dOm = sdesc_add(dOm0, (t % S) * C::kTile);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           mma_ts(tdV, tS + ks * 8 + (ks >= 4 ? 32 : 0), sdesc_add(dOm, ks * 2048), id_kxmn,
@@ -496,7 +507,7 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
         FA_TRACE(16 + t * 8 + 2);
       };
       auto issue_dK = [&](int t, bool acc) {  // dK += dS^T Q_i
-        const uint64_t dQm = sdesc_add(dQm0, (t & 1) * C::kTile);
+        const uint64_t dQm = sdesc_add(dQm0, (t % S) * C::kTile);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
@@ -511,7 +522,7 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
         FA_TRACE(16 + t * 8 + 3);
       };
       auto wait_stage = [&](int t) {
-        return mbar_wait(ctx, &bar_qdo_full[t & 1], (t >> 1) & 1, kBTagQdoFull);
+        return mbar_wait(ctx, &bar_qdo_full[t % S], (t / S) & 1, kBTagQdoFull);
       };
       // S^T(i+1) overwrites P^T(i), which dV(i) reads, and dP^T(i+1) the dP^T(i)
       // the compute warps have turned into dS(i): neither waits for an MMA to
@@ -550,7 +561,7 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
             issue_dK(t, it > 0);
             if constexpr (NO_DQ) {
               mma_commit(bar_dkq_done);
-              mma_commit(&bar_staged[t & 1]);
+              mma_commit(&bar_staged[t % S]);
             } else {
               if (t > 0) {  // dQ of the previous tile has left its columns
                 if (!(ok = mbar_wait(ctx, bar_dq_empty, (t - 1) & 1, kBTagDqEmpty))) break;
@@ -582,6 +593,8 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
             issue_dQ(t);
           }
         }
+        if (!ok) break;
+        mma_commit(bar_kv_free);  // every MMA of this unit: K_j, V_j may be reloaded
         t = t0 + n_it;
       }
       if (!ok) {
@@ -618,7 +631,7 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
       }
       for (int it = 0; it < n_it && ok; ++it) {
         const int t = t0 + it;
-        const int s = t & 1, n = t >> 1;
+        const int s = t % S, n = t / S;
         ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_s_full, t & 1, kBTagSFull) &&
                                          mbar_wait(ctx, &bar_qdo_full[s], n & 1, kBTagQdoFull));
         if (!ok) break;
@@ -817,7 +830,7 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
       bwd_unit(unit, p.BH, nq, bh, j);
       const int i0 = CAUSAL ? j : 0, n_it = nq - i0;
       for (int it = 0; it < n_it && ok; ++it) {
-        const int t = t0 + it, s = t & 1;
+        const int t = t0 + it, s = t % S;
         ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, t & 1, kBTagDkqDone));
         if (!ok) break;
         tc_fence_after();

@@ -6,14 +6,14 @@ j, with its query tiles); its tiles are numbered across units (t), and every
 per-tile barrier phase and stage follows t.  Roles, as in the kernel:
   * producer: hands each unit to the other roles through a two-slot ring (the
     kernel fetches the next unit from a counter); per tile t, Q_t, dO_t, LSE_t,
-    D_t into stage t % 2.  With drain warps (d = 64) it reloads a stage after
-    its "empty" barrier; in the compute-drain layout (d = 128, and every no-dQ
-    instantiation) it frees tile t - 2's stage itself just before reloading it:
-    it waits for the compute warps' staged dQ(t-2) and reduce-adds it (no dQ: it
-    waits for the issuer's commit after dK(t-2)), and frees the last two tiles the
-    same way at the end.
+    D_t into stage t % S (S = 3 stages at d = 64, 2 at d = 128).  With drain
+    warps (d = 64) it reloads a stage after its "empty" barrier; in the
+    compute-drain layout (d = 128, and every no-dQ instantiation) it frees tile
+    t - S's stage itself just before reloading it: it waits for the compute warps'
+    staged dQ(t-S) and reduce-adds it (no dQ: it waits for the issuer's commit
+    after dK(t-S)), and frees the last S tiles the same way at the end.
     K_j and V_j of a unit load after its first tile, once every MMA of the
-    previous unit (the last dK / dQ) has completed;
+    previous unit has completed (the issuer's per-unit commit);
   * issuer (one thread), five MMAs per query tile:
       d = 128:  S^T(t) dP^T(t) [P^T] dV(t) [dS] dK(t) dQ(t)   (dQ in dP^T's columns,
                 so dP^T(t+1) waits until the drain has read dQ(t))
@@ -64,17 +64,19 @@ def bwd_model(units, d: int, seed: int, dropout: bool = False, skip: str = "", n
     first = [sum(units[:u]) for u in range(n_units)]  # global index of each unit's first tile
     M = Machine(seed)
     compute_drain = d == 128 or no_dq  # the kernel's BwdRoles::kComputeDrain
+    S = 3 if d == 64 else 2  # the kernel's BwdCfg::kQStages: tile t sits in stage t % S
     bar_kv = Bar("kv", 2)
-    qdo_full = [Bar(f"qdo_full{s}", 4) for s in range(2)]  # Q, dO, LSE, D
-    qdo_empty = [Bar(f"qdo_empty{s}", 1) for s in range(2)]
+    qdo_full = [Bar(f"qdo_full{s}", 4) for s in range(S)]  # Q, dO, LSE, D
+    qdo_empty = [Bar(f"qdo_empty{s}", 1) for s in range(S)]
     # compute-drain layout: every compute warp staged its dQ part; without dQ, the
     # issuer's commit after dK(t) (a per-stage barrier: a wait on it cannot fall two
     # phases behind, unlike one on dkq_done)
-    staged = [Bar(f"staged{s}", 1 if no_dq else 8) for s in range(2)]
+    staged = [Bar(f"staged{s}", 1 if no_dq else 8) for s in range(S)]
     s_full, dp_full = Bar("s_full", 1), Bar("dp_full", 1)
     p_full, ds_full = Bar("p_full", 8), Bar("ds_full", 8)
     dkq_done, dq_empty = Bar("dkq_done", 1), Bar("dq_empty", 8 if compute_drain else 4)
     stage = Bar("stage", 4)
+    kv_free = Bar("kv_free", 1)  # the issuer's commit after a unit's last MMA
     consumers = 1 + 8 + (0 if compute_drain else 4)  # issuer, compute warps, drain warps
     unit_full = [Bar(f"unit_full{s}", 1) for s in range(2)]
     unit_empty = [Bar(f"unit_empty{s}", consumers) for s in range(2)]
@@ -89,12 +91,12 @@ def bwd_model(units, d: int, seed: int, dropout: bool = False, skip: str = "", n
 
     def free_stage(t):
         """Compute-drain layout: the producer frees tile t's stage."""
-        st = t & 1
+        st = t % S
         if no_dq:
-            yield lambda: staged[st].ready(t >> 1)
+            yield lambda: staged[st].ready(t // S)
             return
         if skip != "staged_wait":
-            yield lambda: staged[st].ready(t >> 1)
+            yield lambda: staged[st].ready(t // S)
         M.read(("Q", st), ("dQ staged", t))  # the reduce-add's read (waited for)
         M.read(("dO", st), ("dQ staged", t))
 
@@ -109,29 +111,31 @@ def bwd_model(units, d: int, seed: int, dropout: bool = False, skip: str = "", n
                 break
             for it in range(units[u]):
                 t = first[u] + it
-                s, n = t & 1, t >> 1
+                s, n = t % S, t // S
                 if compute_drain:
-                    if t >= 2:
-                        yield from free_stage(t - 2)
+                    if t >= S:
+                        yield from free_stage(t - S)
                 elif n > 0:
                     yield lambda s=s, n=n: qdo_empty[s].ready(n - 1)
                 for nm in ("Q", "dO", "L", "Dv"):
                     M.load((nm, s), (nm, t), qdo_full[s])
                 if it == 0:
-                    # K_j, V_j of this unit: after every MMA of the previous one
+                    # K_j, V_j of this unit: after every MMA of the previous one (a
+                    # per-unit barrier: a wait on dkq_done(t-1) could pass early
+                    # with three stages, the producer running that far ahead)
                     if u > 0 and skip != "kv_wait":
-                        yield lambda t=t: dkq_done.ready(t - 1)
+                        yield lambda u=u: kv_free.ready(u - 1)
                     M.load("K", ("K", u), bar_kv)
                     M.load("V", ("V", u), bar_kv)
         T = first[-1] + units[-1]
         if compute_drain:
             if not no_dq or skip == "tail_waits":  # no dQ: the epilogue itself waits for the last dK
-                for t in range(max(T - 2, 0), T):
+                for t in range(max(T - S, 0), T):
                     yield from free_stage(t)
 
     def issuer():
         def stage_ready(t):
-            return lambda: qdo_full[t & 1].ready(t >> 1)
+            return lambda: qdo_full[t % S].ready(t // S)
 
         for u in range(n_units + 1):
             yield from get_unit(u)
@@ -140,29 +144,29 @@ def bwd_model(units, d: int, seed: int, dropout: bool = False, skip: str = "", n
             n_it, t0 = units[u], first[u]
 
             def sT(t):
-                M.mma(0, {"K": ("K", u), ("Q", t & 1): ("Q", t)}, {p: ("S", t) for p in parts("ST")})
+                M.mma(0, {"K": ("K", u), ("Q", t % S): ("Q", t)}, {p: ("S", t) for p in parts("ST")})
                 M.commit(0, s_full)
 
             def dPT(t):
-                M.mma(0, {"V": ("V", u), ("dO", t & 1): ("dO", t)}, {p: ("dP", t) for p in parts("dPT")})
+                M.mma(0, {"V": ("V", u), ("dO", t % S): ("dO", t)}, {p: ("dP", t) for p in parts("dPT")})
                 M.commit(0, dp_full)
 
             def dV(t):
                 it = t - t0
-                reads = {**{p: ("P", t) for p in parts("ST")}, ("dO", t & 1): ("dO", t)}
+                reads = {**{p: ("P", t) for p in parts("ST")}, ("dO", t % S): ("dO", t)}
                 if it > 0:
                     reads["dV"] = (u, it)
                 M.mma(0, reads, {"dV": (u, it + 1)})
 
             def dK(t):
                 it = t - t0
-                reads = {**{p: ("dS", t) for p in parts("dS")}, ("Q", t & 1): ("Q", t)}
+                reads = {**{p: ("dS", t) for p in parts("dS")}, ("Q", t % S): ("Q", t)}
                 if it > 0:
                     reads["dK"] = (u, it)
                 M.mma(0, reads, {"dK": (u, it + 1)})
                 if no_dq:  # without the dQ product, dK(t) closes the tile and frees its stage
                     M.commit(0, dkq_done)
-                    M.commit(0, staged[t & 1])
+                    M.commit(0, staged[t % S])
 
             def dQ(t):
                 cols = parts(dq_cols) if d == 128 else [(dq_cols, 0, q) for q in QUARTERS]
@@ -222,6 +226,7 @@ def bwd_model(units, d: int, seed: int, dropout: bool = False, skip: str = "", n
                     dQ(t)
                     if it + 1 < n_it:
                         dPT(t + 1)
+            M.commit(0, kv_free)
 
     def compute(w, q):
         for u in range(n_units + 1):
@@ -231,7 +236,7 @@ def bwd_model(units, d: int, seed: int, dropout: bool = False, skip: str = "", n
             n_it, t0 = units[u], first[u]
             for it in range(n_it):
                 t = t0 + it
-                s, n = t & 1, t >> 1
+                s, n = t % S, t // S
                 yield lambda t=t, s=s, n=n: s_full.ready(t) and qdo_full[s].ready(n)
                 if dropout:
                     if t > 0 and skip != "draws_wait":
@@ -276,7 +281,7 @@ def bwd_model(units, d: int, seed: int, dropout: bool = False, skip: str = "", n
                 return
             for it in range(units[u]):
                 t = first[u] + it
-                s = t & 1
+                s = t % S
                 yield lambda t=t: dkq_done.ready(t)
                 M.read((dq_cols, 0, q), ("dQ", t))
                 dq_empty.arrive()
