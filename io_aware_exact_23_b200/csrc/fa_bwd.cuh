@@ -30,7 +30,7 @@
 //               after each tile's dS and the producer issues the reduce-add.
 //   producer    (warp 12 / 8) TMA: K_j, V_j once; Q_i, dO_i, LSE_i, D_i per
 //               tile (2 stages)
-//   issuer      (warp 13 / 9) MMAs (one thread), five per query tile:
+//   issuer      (warp 13 / 9) MMAs (one elected lane), five per query tile:
 //                 S^T  = K_j Q_i^T      (smem x smem)      -> TMEM
 //                 dP^T = V_j dO_i^T     (smem x smem)      -> TMEM
 //                 dV  += P^T dO_i       (TMEM x smem)
@@ -361,19 +361,14 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
   if (threadIdx.x == 0) FA_TRACE(0);
 
   // A consumer warp (all lanes) takes unit u from the ring: its index, or -1 (no
-  // more units); take_unit_1 is the same for the issuer's single thread.
+  // more units), broadcast from lane 0 so that the compiler knows it is
+  // warp-uniform.
   auto take_unit = [&](int u, int &unit) -> bool {
     const bool ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_unit_full[u & 1], (u >> 1) & 1, kBTagUnit));
     if (!ok) return false;
-    unit = unit_ring[u & 1];
+    unit = __shfl_sync(0xffffffffu, unit_ring[u & 1], 0);
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar_unit_empty[u & 1]);
-    return true;
-  };
-  auto take_unit_1 = [&](int u, int &unit) -> bool {
-    if (!mbar_wait(ctx, &bar_unit_full[u & 1], (u >> 1) & 1, kBTagUnit)) return false;
-    unit = unit_ring[u & 1];
-    mbar_arrive(&bar_unit_empty[u & 1]);
     return true;
   };
 
@@ -464,7 +459,14 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
     __syncwarp();
   } else if (warp == R::kIssuerWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && !*abort_flag) {
+    // The whole warp runs the issue loop, so that its descriptors and TMEM
+    // addresses are warp-uniform values; one elected lane issues each MMA and
+    // commit (the warp-wide forms in ptx.cuh).
+    const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+    if (__all_sync(0xffffffffu, *abort_flag == 0)) {
+      auto wait = [&](uint64_t *bar, int parity, int tag) {
+        return __all_sync(0xffffffffu, mbar_wait(ctx, bar, static_cast<uint32_t>(parity), tag));
+      };
       constexpr uint32_t id_ss = make_idesc_bf16(128, 128, 0, 0);     // S^T, dP^T
       constexpr uint32_t id_kxmn = make_idesc_bf16(128, D, 0, 1);     // dV (A in TMEM), dK
       constexpr uint32_t id_mnmn = make_idesc_bf16(128, D, 1, 1);     // dQ
@@ -474,8 +476,8 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
       const uint64_t dSk = make_sdesc(smem_u32(sdS), 16, 1024), dSm = make_sdesc(smem_u32(sdS), 16384, 1024);
       const uint64_t dQk0 = make_sdesc(smem_u32(sQ), 16, 1024), dQm0 = make_sdesc(smem_u32(sQ), 16384, 1024);
       const uint64_t dOk0 = make_sdesc(smem_u32(sdO), 16, 1024), dOm0 = make_sdesc(smem_u32(sdO), 16384, 1024);
-      const uint32_t tS = tmem + C::kColS, tdP = tmem + C::kColdP, tdK = tmem + C::kColdK;
-      const uint32_t tdV = tmem + C::kColdV, tdQ = tmem + C::kColdQ;
+      const uint32_t tS = tm + C::kColS, tdP = tm + C::kColdP, tdK = tm + C::kColdK;
+      const uint32_t tdV = tm + C::kColdV, tdQ = tm + C::kColdQ;
       // t: the tile's index over all units (its stage is t % 2); acc: accumulate
       // into dK / dV (false for a unit's first query tile).
       auto issue_sT = [&](int t) {  // S^T = K_j Q_i^T
@@ -483,60 +485,60 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_ss(tS, sdesc_add(dKk, off), sdesc_add(dQk, off), id_ss, ks > 0);
+          mma_ss_w(tS, sdesc_add(dKk, off), sdesc_add(dQk, off), id_ss, ks > 0);
         }
-        mma_commit(bar_s_full);
-        FA_TRACE(16 + t * 8 + 0);
+        mma_commit_w(bar_s_full);
+        if (lane == 0) FA_TRACE(16 + t * 8 + 0);
       };
       auto issue_dPT = [&](int t) {  // dP^T = V_j dO_i^T
         const uint64_t dOk = sdesc_add(dOk0, (t % S) * C::kTile);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_ss(tdP, sdesc_add(dVk, off), sdesc_add(dOk, off), id_ss, ks > 0);
+          mma_ss_w(tdP, sdesc_add(dVk, off), sdesc_add(dOk, off), id_ss, ks > 0);
         }
-        mma_commit(bar_dp_full);
-        FA_TRACE(16 + t * 8 + 1);
+        mma_commit_w(bar_dp_full);
+        if (lane == 0) FA_TRACE(16 + t * 8 + 1);
       };
       auto issue_dV = [&](int t, bool acc) {  // dV += P^T dO_i; P^T of query columns 64w.. at S^T columns 64w..64w+31
         const uint64_t dOm = sdesc_add(dOm0, (t % S) * C::kTile);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_ts(tdV, tS + ks * 8 + (ks >= 4 ? 32 : 0), sdesc_add(dOm, ks * 2048), id_kxmn,
+          mma_ts_w(tdV, tS + ks * 8 + (ks >= 4 ? 32 : 0), sdesc_add(dOm, ks * 2048), id_kxmn,
                  (acc || ks > 0) ? 1u : 0u);
-        FA_TRACE(16 + t * 8 + 2);
+        if (lane == 0) FA_TRACE(16 + t * 8 + 2);
       };
       auto issue_dK = [&](int t, bool acc) {  // dK += dS^T Q_i
         const uint64_t dQm = sdesc_add(dQm0, (t % S) * C::kTile);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_ss(tdK, sdesc_add(dSk, off), sdesc_add(dQm, ks * 2048), id_kxmn, (acc || ks > 0) ? 1u : 0u);
+          mma_ss_w(tdK, sdesc_add(dSk, off), sdesc_add(dQm, ks * 2048), id_kxmn, (acc || ks > 0) ? 1u : 0u);
         }
       };
       auto issue_dQ = [&](int t) {  // dQ_i = dS K_j; the dQ drain releases the Q/dO stage after staging through it
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_ss(tdQ, sdesc_add(dSm, ks * 2048), sdesc_add(dKm, ks * 2048), id_mnmn, ks > 0);
-        mma_commit(bar_dkq_done);
-        FA_TRACE(16 + t * 8 + 3);
+          mma_ss_w(tdQ, sdesc_add(dSm, ks * 2048), sdesc_add(dKm, ks * 2048), id_mnmn, ks > 0);
+        mma_commit_w(bar_dkq_done);
+        if (lane == 0) FA_TRACE(16 + t * 8 + 3);
       };
       auto wait_stage = [&](int t) {
-        return mbar_wait(ctx, &bar_qdo_full[t % S], (t / S) & 1, kBTagQdoFull);
+        return wait(&bar_qdo_full[t % S], (t / S) & 1, kBTagQdoFull);
       };
       // S^T(i+1) overwrites P^T(i), which dV(i) reads, and dP^T(i+1) the dP^T(i)
       // the compute warps have turned into dS(i): neither waits for an MMA to
-      // complete, since one thread issues them all and the pipe runs them in order.
+      // complete, since one lane issues them all and the pipe runs them in order.
       bool ok = true;
       int t = 0;  // query tiles issued so far, over all units
       for (int u = 0; ok; ++u) {
         int unit;
-        if (!(ok = take_unit_1(u, unit))) break;
+        if (!(ok = take_unit(u, unit))) break;
         if (unit < 0) break;
         int bh, j;
         bwd_unit(unit, p.BH, nq, bh, j);
         const int n_it = nq - (CAUSAL ? j : 0), t0 = t;
-        if (!(ok = mbar_wait(ctx, bar_kv, u & 1, kBTagKV))) break;
+        if (!(ok = wait(bar_kv, u & 1, kBTagKV))) break;
         if (NO_DQ || D == 64) {
           // Order S^T(0) dP^T(0) | dV(i) S^T(i+1) dK(i) [dQ(i)] dP^T(i+1) | ...: the
           // next tile's S^T goes in ahead of dK(i) (and dQ(i), which has columns of
@@ -548,7 +550,7 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
           issue_dPT(t0);
           for (int it = 0; it < n_it && ok; ++it) {
             t = t0 + it;
-            if (!(ok = mbar_wait(ctx, bar_p_full, t & 1, kBTagPFull))) break;
+            if (!(ok = wait(bar_p_full, t & 1, kBTagPFull))) break;
             tc_fence_after();
             issue_dV(t, it > 0);
             if (it + 1 < n_it) {
@@ -556,15 +558,15 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
               tc_fence_after();
               issue_sT(t + 1);
             }
-            if (!(ok = mbar_wait(ctx, bar_ds_full, t & 1, kBTagDsFull))) break;
+            if (!(ok = wait(bar_ds_full, t & 1, kBTagDsFull))) break;
             tc_fence_after();
             issue_dK(t, it > 0);
             if constexpr (NO_DQ) {
-              mma_commit(bar_dkq_done);
-              mma_commit(&bar_staged[t % S]);
+              mma_commit_w(bar_dkq_done);
+              mma_commit_w(&bar_staged[t % S]);
             } else {
               if (t > 0) {  // dQ of the previous tile has left its columns
-                if (!(ok = mbar_wait(ctx, bar_dq_empty, (t - 1) & 1, kBTagDqEmpty))) break;
+                if (!(ok = wait(bar_dq_empty, (t - 1) & 1, kBTagDqEmpty))) break;
                 tc_fence_after();
               }
               issue_dQ(t);
@@ -580,25 +582,25 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
             tc_fence_after();
             issue_sT(t);
             if (t > 0) {
-              if (!(ok = mbar_wait(ctx, bar_dq_empty, (t - 1) & 1, kBTagDqEmpty))) break;
+              if (!(ok = wait(bar_dq_empty, (t - 1) & 1, kBTagDqEmpty))) break;
               tc_fence_after();
             }
             issue_dPT(t);
-            if (!(ok = mbar_wait(ctx, bar_p_full, t & 1, kBTagPFull))) break;
+            if (!(ok = wait(bar_p_full, t & 1, kBTagPFull))) break;
             tc_fence_after();
             issue_dV(t, it > 0);
-            if (!(ok = mbar_wait(ctx, bar_ds_full, t & 1, kBTagDsFull))) break;
+            if (!(ok = wait(bar_ds_full, t & 1, kBTagDsFull))) break;
             tc_fence_after();
             issue_dK(t, it > 0);
             issue_dQ(t);
           }
         }
         if (!ok) break;
-        mma_commit(bar_kv_free);  // every MMA of this unit: K_j, V_j may be reloaded
+        mma_commit_w(bar_kv_free);  // every MMA of this unit: K_j, V_j may be reloaded
         t = t0 + n_it;
       }
       if (!ok) {
-        mma_commit(bar_drain);
+        mma_commit_w(bar_drain);
         mbar_drain(bar_drain, 0);
       }
     }

@@ -21,7 +21,7 @@
 //              A thread holds its row's LSE and D in registers.
 //   warp  8    TMA producer: Q_i and dO_i once, then K_0, V_0, K_1, V_1, ...
 //              through a ring of single-tile slots.
-//   warp  9    MMA issuer (one thread) and TMEM owner.  Per key tile it issues
+//   warp  9    MMA issuer (one elected lane) and TMEM owner.  Per key tile it issues
 //              S(j+1) before dQ(j), so the compute warps start on tile j+1's
 //              exponentials while dQ(j) and dP(j+1) run.
 // A slot is released by the MMA that reads its tile last: V_j by dP(j), K_j by
@@ -193,23 +193,29 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else if (warp == C::kIssuerWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && !*abort_flag) {
+    // The whole warp runs the issue loop (warp-uniform descriptors and TMEM
+    // addresses); one elected lane issues each MMA and commit.
+    const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+    if (__all_sync(0xffffffffu, *abort_flag == 0)) {
+      auto wait = [&](uint64_t *bar, int parity, int tag) {
+        return __all_sync(0xffffffffu, mbar_wait(ctx, bar, static_cast<uint32_t>(parity), tag));
+      };
       constexpr uint32_t id_ss = make_idesc_bf16(128, 128, 0, 0);  // S, dP (both operands K-major)
       constexpr uint32_t id_dq = make_idesc_bf16(128, D, 0, 1);    // dQ: A = dS (TMEM), B = K_j MN-major
       const uint64_t dQk = make_sdesc(smem_u32(sQ), 16, 1024);
       const uint64_t dOk = make_sdesc(smem_u32(sdO), 16, 1024);
       const uint64_t kvk0 = make_sdesc(smem_u32(sKV), 16, 1024);     // slot 0, K-major view
       const uint64_t kvm0 = make_sdesc(smem_u32(sKV), 16384, 1024);  // slot 0, MN-major view
-      const uint32_t tdP = tmem + C::kColdP, tdQ = tmem + C::kColdQ;
+      const uint32_t tdP = tm + C::kColdP, tdQ = tm + C::kColdQ;
       auto issue_S = [&](int j) {  // S(j) = Q_i K_j^T -> S buffer j & 1
         const uint64_t kd = sdesc_add(kvk0, dq_slot(2 * j, C::kSlots) * C::kTile);
-        const uint32_t tS = tmem + C::kColS + 128 * (j & 1);
+        const uint32_t tS = tm + C::kColS + 128 * (j & 1);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_ss(tS, sdesc_add(dQk, off), sdesc_add(kd, off), id_ss, ks > 0);
+          mma_ss_w(tS, sdesc_add(dQk, off), sdesc_add(kd, off), id_ss, ks > 0);
         }
-        mma_commit(&bar_s_full[j & 1]);
+        mma_commit_w(&bar_s_full[j & 1]);
       };
       auto issue_dP = [&](int j) {  // dP(j) = dO_i V_j^T; V_j's slot is free once it completes
         const int sv = dq_slot(2 * j + 1, C::kSlots);
@@ -217,25 +223,25 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_ss(tdP, sdesc_add(dOk, off), sdesc_add(vd, off), id_ss, ks > 0);
+          mma_ss_w(tdP, sdesc_add(dOk, off), sdesc_add(vd, off), id_ss, ks > 0);
         }
-        mma_commit(bar_dp_full);
-        mma_commit(&bar_kv_empty[sv]);
+        mma_commit_w(bar_dp_full);
+        mma_commit_w(&bar_kv_empty[sv]);
       };
       auto issue_dQ = [&](int j) {  // dQ += dS(j) K_j; K_j's slot is free once it completes
         const int sk = dq_slot(2 * j, C::kSlots);
         const uint64_t km = sdesc_add(kvm0, sk * C::kTile);
-        const uint32_t tS = tmem + C::kColS + 128 * (j & 1);
+        const uint32_t tS = tm + C::kColS + 128 * (j & 1);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_ts(tdQ, tS + ks * 8 + (ks >= 4 ? 32 : 0), sdesc_add(km, ks * 2048), id_dq,
+          mma_ts_w(tdQ, tS + ks * 8 + (ks >= 4 ? 32 : 0), sdesc_add(km, ks * 2048), id_dq,
                  (j > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(&bar_kv_empty[sk]);
+        mma_commit_w(&bar_kv_empty[sk]);
       };
       auto wait_kv = [&](int idx) {
-        return mbar_wait(ctx, &bar_kv_full[dq_slot(idx, C::kSlots)], dq_phase(idx, C::kSlots), kQTagKvFull);
+        return wait(&bar_kv_full[dq_slot(idx, C::kSlots)], static_cast<int>(dq_phase(idx, C::kSlots)), kQTagKvFull);
       };
-      bool ok = mbar_wait(ctx, bar_qdo, 0, kQTagQdo) && wait_kv(0) && wait_kv(1);
+      bool ok = wait(bar_qdo, 0, kQTagQdo) && wait_kv(0) && wait_kv(1);
       if (ok) {
         tc_fence_after();
         issue_S(0);
@@ -248,7 +254,7 @@ __global__ void __launch_bounds__(320, 1)
           tc_fence_after();
           issue_S(j + 1);
         }
-        ok = mbar_wait(ctx, bar_ds_full, j & 1, kQTagDsFull);
+        ok = wait(bar_ds_full, j & 1, kQTagDsFull);
         if (!ok) break;
         tc_fence_after();
         issue_dQ(j);
@@ -260,10 +266,10 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       if (ok) {
-        mma_commit(bar_dq_done);
+        mma_commit_w(bar_dq_done);
       } else {
-        // Let every MMA this thread issued finish before TMEM is released.
-        mma_commit(bar_drain);
+        // Let every MMA this warp issued finish before TMEM is released.
+        mma_commit_w(bar_drain);
         mbar_drain(bar_drain, 0);
       }
     }

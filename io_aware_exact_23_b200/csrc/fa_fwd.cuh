@@ -15,7 +15,7 @@
 //              pipe runs the other tile's PV and next S.  The two warps that
 //              share rows exchange their half-row maxima through smem.
 //   warp  8    TMA producer: Q0, Q1 once, then K / V tiles through a smem ring.
-//   warp  9    MMA issuer for tile 0 (one thread); warp 10 for tile 1.  Two
+//   warp  9    MMA issuer for tile 0 (one elected lane); warp 10 for tile 1.  Two
 //              independent issuers let the pipe take whichever tile is ready.
 // A K/V ring stage is released when both issuers' MMAs that read it completed.
 //
@@ -219,20 +219,14 @@ __global__ void __launch_bounds__(352, 1)
     n0 = CAUSAL ? min(2 * u + 1, n_kv_all) : n_kv_all;
     n1 = CAUSAL ? min(2 * u + 2, n_kv_all) : n_kv_all;
   };
-  // A consumer warp (all lanes) takes unit i from the ring; take_unit_1 is the
-  // same for an issuer's single thread.  -1: no more units.
+  // A consumer warp (all lanes) takes unit i from the ring (-1: no more units).
+  // The value is broadcast from lane 0, so the compiler knows it is warp-uniform.
   auto take_unit = [&](int i, int &unit) -> bool {
     const bool ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_unit_full[i & 1], (i >> 1) & 1, kTagUnit));
     if (!ok) return false;
-    unit = unit_ring[i & 1];
+    unit = __shfl_sync(0xffffffffu, unit_ring[i & 1], 0);
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar_unit_empty[i & 1]);
-    return true;
-  };
-  auto take_unit_1 = [&](int i, int &unit) -> bool {
-    if (!mbar_wait(ctx, &bar_unit_full[i & 1], (i >> 1) & 1, kTagUnit)) return false;
-    unit = unit_ring[i & 1];
-    mbar_arrive(&bar_unit_empty[i & 1]);
     return true;
   };
 
@@ -302,87 +296,95 @@ __global__ void __launch_bounds__(352, 1)
     __syncwarp();
   } else if (warp == C::kIssuerWarp || warp == C::kIssuerWarp + 1) {
     // ------------------------------------------------------------ MMA issuers
-    const int k = warp - C::kIssuerWarp;  // query tile owned by this issuer
-    if (lane == 0 && !*abort_flag) {
+    // The whole warp runs the issue loop (waits, unit decode, descriptors), so
+    // that every value it computes is warp-uniform; one elected lane issues each
+    // MMA and commit.  Run from a single lane, the same loop took about 100 SM
+    // cycles per MMA while the softmax warps kept the sub-partition busy.
+    const int k = __shfl_sync(0xffffffffu, warp, 0) - C::kIssuerWarp;  // query tile owned by this issuer
+    const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+    if (__all_sync(0xffffffffu, *abort_flag == 0)) {
       constexpr uint32_t idesc_qk = FP8 ? make_idesc_e4m3(128, 128, 0, 0) : make_idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = FP8 ? make_idesc_e4m3(128, D, 0, 1) : make_idesc_bf16(128, D, 0, 1);
       // Base descriptors: Q_k (K-major), ring stage 0 as K (K-major) and as V (MN-major).
       const uint64_t q_desc = make_sdesc(smem_u32(sQ + k * C::kTileBytes), 16, 1024);
       const uint64_t k_desc0 = make_sdesc(smem_u32(sKV), 16, 1024);
       const uint64_t v_desc0 = make_sdesc(smem_u32(sKV), 16384, 1024);
-      const uint32_t tS = tmem + 128 * k;
-      const uint32_t tO = tmem + 256 + k * D;
+      const uint32_t tS = tm + 128 * k;
+      const uint32_t tO = tm + 256 + k * D;
       bool ok = true;
       int gb = 0;  // K/V loads of the previous units
       int cs = 0;  // this tile's KV steps in the previous units
+      auto wait = [&](uint64_t *bar, int parity, int tag) {
+        return __all_sync(0xffffffffu, mbar_wait(ctx, bar, static_cast<uint32_t>(parity), tag));
+      };
       for (int ui = 0; ok; ++ui) {
         int unit;
-        if (!(ok = take_unit_1(ui, unit))) break;
+        if (!(ok = take_unit(ui, unit))) break;
         if (unit < 0) break;
         int bh, u, n0, n_kv;
         decode(unit, bh, u);
         steps(u, n0, n_kv);
         const int n_k = (k == 0) ? n0 : n_kv;
-        if (!(ok = mbar_wait(ctx, &bar_q[k], ui & 1, kTagQ))) break;
+        if (!(ok = wait(&bar_q[k], ui & 1, kTagQ))) break;
         for (int j = 0; j < n_kv && ok; ++j) {
           const int iK = gb + kv_idx_k(j), sK = iK % C::kStages;
           const int iV = gb + kv_idx_v(j, n_kv), sV = iV % C::kStages;
           // Arrivals on kv_empty must follow the matching kv_full phase, so even
           // a tile that skips K_j / V_j (causal tile 0 past its diagonal) waits.
-          ok = mbar_wait(ctx, &bar_kv_full[sK], (iK / C::kStages) & 1, kTagKvFull);
+          ok = wait(&bar_kv_full[sK], (iK / C::kStages) & 1, kTagKvFull);
           if (!ok) break;
           if (j >= n_k) {
-            mbar_arrive(&bar_kv_empty[sK]);
-            ok = mbar_wait(ctx, &bar_kv_full[sV], (iV / C::kStages) & 1, kTagKvFull);
-            if (ok) mbar_arrive(&bar_kv_empty[sV]);
+            if (lane == 0) mbar_arrive(&bar_kv_empty[sK]);
+            ok = wait(&bar_kv_full[sV], (iV / C::kStages) & 1, kTagKvFull);
+            if (ok && lane == 0) mbar_arrive(&bar_kv_empty[sV]);
             continue;
           }
           // S_k aliases P_k, which the previous PV_k reads.  Both MMAs come from
-          // this thread and the tensor pipe runs them in issue order, so S_k is
-          // issued right behind PV_k without waiting for it to complete.
+          // this warp's elected lane and the tensor pipe runs them in issue order,
+          // so S_k is issued right behind PV_k without waiting for it to complete.
           const uint64_t k_desc = sdesc_add(k_desc0, sK * C::kTileBytes);
           // One MMA per 32-byte K slice of the 128-byte swizzled rows (16 bf16 or 32 e4m3).
 #pragma unroll
           for (int ks = 0; ks < D * C::kElemBytes / 32; ++ks) {
             const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
             if constexpr (FP8)
-              mma_ss_f8(tS, sdesc_add(q_desc, off), sdesc_add(k_desc, off), idesc_qk, ks > 0);
+              mma_ss_f8_w(tS, sdesc_add(q_desc, off), sdesc_add(k_desc, off), idesc_qk, ks > 0);
             else
-              mma_ss(tS, sdesc_add(q_desc, off), sdesc_add(k_desc, off), idesc_qk, ks > 0);
+              mma_ss_w(tS, sdesc_add(q_desc, off), sdesc_add(k_desc, off), idesc_qk, ks > 0);
           }
-          mma_commit(&bar_s_full[k]);
-          mma_commit(&bar_kv_empty[sK]);
-          if (j == n_k - 1) mma_commit(&bar_q_free[k]);  // Q_k is not read again in this unit
-          FA_TRACE(16 + k * 256 + 4 * j + 0);
-          ok = mbar_wait(ctx, &bar_kv_full[sV], (iV / C::kStages) & 1, kTagKvFull);
-          if (ok) ok = mbar_wait(ctx, &bar_p_full[k], (cs + j) & 1, kTagPFull);
+          mma_commit_w(&bar_s_full[k]);
+          mma_commit_w(&bar_kv_empty[sK]);
+          if (j == n_k - 1) mma_commit_w(&bar_q_free[k]);  // Q_k is not read again in this unit
+          if (lane == 0) FA_TRACE(16 + k * 256 + 4 * j + 0);
+          ok = wait(&bar_kv_full[sV], (iV / C::kStages) & 1, kTagKvFull);
+          if (ok) ok = wait(&bar_p_full[k], (cs + j) & 1, kTagPFull);
           if (!ok) break;
           tc_fence_after();
-          FA_TRACE(16 + k * 256 + 4 * j + 2);
+          if (lane == 0) FA_TRACE(16 + k * 256 + 4 * j + 2);
           const uint64_t v_desc = sdesc_add(v_desc0, sV * C::kTileBytes);
           // K steps over the 128 keys: 16 (bf16) or 32 (e4m3) keys, 8 TMEM columns of P
           // and 16 or 32 rows of V each; P of keys 64h.. starts at column 64h.
           if constexpr (FP8) {
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-              mma_ts_f8(tO, tS + ks * 8 + (ks >= 2 ? 48 : 0), sdesc_add(v_desc, ks * 4096), idesc_pv,
-                        (j > 0 || ks > 0) ? 1u : 0u);
+              mma_ts_f8_w(tO, tS + ks * 8 + (ks >= 2 ? 48 : 0), sdesc_add(v_desc, ks * 4096), idesc_pv,
+                          (j > 0 || ks > 0) ? 1u : 0u);
           } else {
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
-              mma_ts(tO, tS + ks * 8 + (ks >= 4 ? 32 : 0), sdesc_add(v_desc, ks * 2048), idesc_pv,
-                     (j > 0 || ks > 0) ? 1u : 0u);
+              mma_ts_w(tO, tS + ks * 8 + (ks >= 4 ? 32 : 0), sdesc_add(v_desc, ks * 2048), idesc_pv,
+                       (j > 0 || ks > 0) ? 1u : 0u);
           }
-          mma_commit(&bar_pv_done[k]);
-          mma_commit(&bar_kv_empty[sV]);
-          FA_TRACE(16 + k * 256 + 4 * j + 1);
+          mma_commit_w(&bar_pv_done[k]);
+          mma_commit_w(&bar_kv_empty[sV]);
+          if (lane == 0) FA_TRACE(16 + k * 256 + 4 * j + 1);
         }
         gb += 2 * n_kv;
         cs += n_k;
       }
       if (!ok) {
-        // Let every MMA this thread issued finish before TMEM is released.
-        mma_commit(&bar_drain[k]);
+        // Let every MMA this warp issued finish before TMEM is released.
+        mma_commit_w(&bar_drain[k]);
         mbar_drain(&bar_drain[k], 0);
       }
     }
