@@ -142,10 +142,11 @@ int fa_fwd_fp8(const void *q8, const void *k8, const void *v8,
  *   seed    64-bit key of the Philox4x32-10 generator (Salmon et al., SC 2011);
  *   offset  counter word 3 (e.g. the training step): a new mask per value.
  * Mask: for head bh = b*H + h, query row i and key j, the generator's counter is
- * (i, j >> 3, bh, offset) and its key (seed & 0xffffffff, seed >> 32); the
- * 16-bit draw of key j is half (j & 1) of output word ((j & 7) >> 1); key j is
- * kept for row i iff the draw is >= T = floor(rate * 65536).  Then
- *   O_i = sum_j P_ij * keep_ij * 65536/(65536 - T) * V_j
+ * (i, j >> 4, bh, offset) and its key (seed & 0xffffffff, seed >> 32); the
+ * 8-bit draw of key j is byte (j & 3) of output word ((j & 15) >> 2); key j is
+ * kept for row i iff the draw is >= T = floor(rate * 256) (the rate takes steps
+ * of 1/256).  Then
+ *   O_i = sum_j P_ij * keep_ij * 256/(256 - T) * V_j
  * with P = softmax(scale * Q K^T [+ causal mask]); lse is that of P, without
  * dropout.  The mask is never stored: fa_bwd_dropout regenerates it.
  */
@@ -158,7 +159,7 @@ int fa_fwd_dropout(const void *q, const void *k, const void *v, void *o,
  * Backward pass of fa_fwd_dropout, given the same rate, seed and offset (and
  * that call's o, o_lo, lse): dV = (P o Z)^T dO, dP = Z o (dO V^T),
  * dS = P o (dP - D) with D_i = rowsum(dO_i o O_i), dQ = scale dS K,
- * dK = scale dS^T Q, where Z = keep * 65536/(65536 - T).  Workspace, layout and
+ * dK = scale dS^T Q, where Z = keep * 256/(256 - T).  Workspace, layout and
  * errors as fa_bwd_ex (without events).
  */
 int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o,

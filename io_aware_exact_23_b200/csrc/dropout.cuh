@@ -9,10 +9,10 @@
 // key, and advances the key by the two Weyl increments.
 //
 // Mask layout: for head bh, query row i and key j the counter is
-// (i, j >> 3, bh, offset), the key is the 64-bit seed (low word, high word);
-// the 16-bit draw of key j is half (j & 1) of output word ((j & 7) >> 1), and
-// the key is kept iff the draw is >= T = floor(rate * 65536).  Kept entries
-// are scaled by 65536 / (65536 - T).
+// (i, j >> 4, bh, offset), the key is the 64-bit seed (low word, high word);
+// the 8-bit draw of key j is byte (j & 3) of output word ((j & 15) >> 2), so
+// one call serves 16 keys, and the key is kept iff the draw is >= T =
+// floor(rate * 256).  Kept entries are scaled by 256 / (256 - T).
 #pragma once
 
 #include <cstdint>
@@ -20,11 +20,11 @@
 namespace fa {
 
 struct DropoutParams {
-  uint32_t T;        // drop a key when its 16-bit draw is below T
+  uint32_t T;        // drop a key when its 8-bit draw is below T
   uint32_t seed_lo;  // Philox key
   uint32_t seed_hi;
   uint32_t offset;   // counter word 3 (e.g. the training step)
-  float inv_keep;    // 65536 / (65536 - T)
+  float inv_keep;    // 256 / (256 - T)
 };
 
 __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
@@ -39,18 +39,18 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
   return c;
 }
 
-// The four output words for query row i and keys 8*jblk .. 8*jblk+7.
+// The four output words for query row i and keys 16*jblk .. 16*jblk+15.
 __device__ __forceinline__ uint4 dropout_words(const DropoutParams &dp, uint32_t i, uint32_t jblk, uint32_t bh) {
   return philox4x32_10(make_uint4(i, jblk, bh, dp.offset), dp.seed_lo, dp.seed_hi);
 }
 
-// Keep bits of keys 8*jblk + t (bit t), t = 0..7.
-__device__ __forceinline__ uint32_t dropout_keep8(const DropoutParams &dp, uint32_t i, uint32_t jblk, uint32_t bh) {
+// Keep bits of keys 16*jblk + t (bit t), t = 0..15.
+__device__ __forceinline__ uint32_t dropout_keep16(const DropoutParams &dp, uint32_t i, uint32_t jblk, uint32_t bh) {
   const uint4 w = dropout_words(dp, i, jblk, bh);
   const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
   uint32_t bits = 0;
 #pragma unroll
-  for (int t = 0; t < 8; ++t) bits |= static_cast<uint32_t>(((ws[t >> 1] >> (16 * (t & 1))) & 0xFFFFu) >= dp.T) << t;
+  for (int t = 0; t < 16; ++t) bits |= static_cast<uint32_t>(((ws[t >> 2] >> (8 * (t & 3))) & 0xFFu) >= dp.T) << t;
   return bits;
 }
 

@@ -164,13 +164,13 @@ cudaError_t fwd_set_attribute() {
 // Returns false for a rate outside [0, 1).
 bool dropout_params(float rate, unsigned long long seed, unsigned int offset, fa::DropoutParams *dp) {
   if (!std::isfinite(rate) || rate < 0.f || rate >= 1.f) return false;
-  const double t = std::floor(static_cast<double>(rate) * 65536.0);
-  if (t >= 65536.0) return false;
+  const double t = std::floor(static_cast<double>(rate) * 256.0);
+  if (t >= 256.0) return false;
   dp->T = static_cast<uint32_t>(t);
   dp->seed_lo = static_cast<uint32_t>(seed & 0xffffffffull);
   dp->seed_hi = static_cast<uint32_t>(seed >> 32);
   dp->offset = offset;
-  dp->inv_keep = static_cast<float>(65536.0 / (65536.0 - t));
+  dp->inv_keep = static_cast<float>(256.0 / (256.0 - t));
   return true;
 }
 
@@ -265,18 +265,18 @@ int fwd_counter(DeviceState *ds, int seq, cudaStream_t s, int **out) {
   return FA_OK;
 }
 
-// Dropout mask writer: one thread per (head, query row, 8-key block).
+// Dropout mask writer: one thread per (head, query row, 16-key block).
 __global__ void fa_dropout_mask_kernel(uint8_t *mask, long BH, int N, fa::DropoutParams dp) {
-  const long nblk = (N + 7) / 8;
+  const long nblk = (N + 15) / 16;
   const long total = BH * N * nblk;
   for (long t = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
        t += static_cast<long>(gridDim.x) * blockDim.x) {
     const long jb = t % nblk, row = t / nblk;
     const long i = row % N, bh = row / N;
-    const uint32_t bits = fa::dropout_keep8(dp, static_cast<uint32_t>(i), static_cast<uint32_t>(jb),
-                                            static_cast<uint32_t>(bh));
-    uint8_t *out = mask + row * N + jb * 8;
-    for (int u = 0; u < 8 && jb * 8 + u < N; ++u) out[u] = static_cast<uint8_t>((bits >> u) & 1u);
+    const uint32_t bits = fa::dropout_keep16(dp, static_cast<uint32_t>(i), static_cast<uint32_t>(jb),
+                                             static_cast<uint32_t>(bh));
+    uint8_t *out = mask + row * N + jb * 16;
+    for (int u = 0; u < 16 && jb * 16 + u < N; ++u) out[u] = static_cast<uint8_t>((bits >> u) & 1u);
   }
 }
 

@@ -641,8 +641,9 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
         if (threadIdx.x == 0) FA_TRACE(16 + t * 8 + 4);
         // Dropout: keep bit cc for query i*128 + 64w + cc and this thread's key.
         // The generator's counter blocks run along keys, so the warp draws the
-        // 64 x 32 block together (eight calls per lane) and transposes it through
-        // its own rows of the dS tile, free once the previous tile's dK / dQ are done.
+        // 64 x 32 block together (four calls per lane, 16 keys each) and transposes
+        // it through its own rows of the dS tile, free once the previous tile's
+        // dK / dQ are done.
         uint64_t keep = ~0ull;
         if constexpr (DROPOUT) {
           if (t > 0) ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, (t - 1) & 1, kBTagDkqDone));
@@ -650,17 +651,17 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
           int bh, j;
           bwd_unit(unit, p.BH, nq, bh, j);
           const int i = (CAUSAL ? j : 0) + it;
-          const uint32_t slot = smem_u32(sdS) + w * 16384 + (warp & 3) * 4096;  // [64 queries][32 keys] u16
-          const int b = lane & 3;
-          const uint32_t jblk = static_cast<uint32_t>(j * 128 + (warp & 3) * 32) / 8 + b;
+          const uint32_t slot = smem_u32(sdS) + w * 16384 + (warp & 3) * 4096;  // [64 queries][32 keys] u8
+          const int b = lane & 1;
+          const uint32_t jblk = static_cast<uint32_t>(j * 128 + (warp & 3) * 32) / 16 + b;
 #pragma unroll 1
-          for (int q8 = 0; q8 < 8; ++q8) {
-            const int ii = (lane >> 2) + 8 * q8;
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int ii = (lane >> 1) + 16 * q4;
             const uint4 wv = dropout_words(p.drop, i * 128 + 64 * w + ii, jblk, bh);
-            st_shared_v4(slot + (ii * 32 + 8 * b) * 2, wv.x, wv.y, wv.z, wv.w);
+            st_shared_v4(slot + ii * 32 + 16 * b, wv.x, wv.y, wv.z, wv.w);
           }
           __syncwarp();
-          const uint16_t *draws = reinterpret_cast<const uint16_t *>(sdS + w * 16384 + (warp & 3) * 4096);
+          const uint8_t *draws = reinterpret_cast<const uint8_t *>(sdS + w * 16384 + (warp & 3) * 4096);
           keep = 0;
   #pragma unroll
           for (int ii = 0; ii < 64; ++ii) keep |= static_cast<uint64_t>(draws[ii * 32 + lane] >= p.drop.T) << ii;

@@ -435,14 +435,14 @@ __global__ void __launch_bounds__(352, 1)
               if (cc >= nv) s[cc] = __float_as_uint(-INFINITY);
           }
           // Dropout: keep bit cc for key j*128 + 64h + cc of query row qt*128 + r,
-          // eight keys per generator call (the counter's key block).
+          // sixteen keys per generator call (the counter's key block).
           uint64_t keep = ~0ull;
           if constexpr (DROPOUT) {
             keep = 0;
-            const uint32_t jb0 = static_cast<uint32_t>(j * 128 + 64 * h) >> 3;
+            const uint32_t jb0 = static_cast<uint32_t>(j * 128 + 64 * h) >> 4;
   #pragma unroll
-            for (int t = 0; t < 8; ++t)
-              keep |= static_cast<uint64_t>(dropout_keep8(p.drop, qt * 128 + r, jb0 + t, bh)) << (8 * t);
+            for (int t = 0; t < 4; ++t)
+              keep |= static_cast<uint64_t>(dropout_keep16(p.drop, qt * 128 + r, jb0 + t, bh)) << (16 * t);
           }
           // Half-row max as a shallow tree (eight independent chains of four).
           float mq[8];

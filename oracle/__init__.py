@@ -176,12 +176,12 @@ def ref_dkdv_rows(q, k, v, dO, scale: float, causal: bool, head: int, key_rows, 
 # ------------------------------------------------------------------ dropout
 
 def dropout_threshold(rate: float) -> int:
-    """T = floor(rate * 65536), with the rate as the 32-bit float the C interface takes:
-    a key is dropped when its 16-bit draw is below T."""
+    """T = floor(rate * 256), with the rate as the 32-bit float the C interface takes:
+    a key is dropped when its 8-bit draw is below T."""
     r = float(np.float32(rate))
     if not (0.0 <= r < 1.0):
         raise ValueError("dropout rate must be in [0, 1)")
-    return int(np.floor(r * 65536.0))
+    return int(np.floor(r * 256.0))
 
 
 def philox4x32_10(counter, key):

@@ -15,16 +15,17 @@
  * the key, and then bumps the key by the two Weyl constants.
  *
  * Mask: for head bh = b*H + h, query row i and key j, the counter is
- * (i, j >> 3, bh, offset) and the key (seed & 0xffffffff, seed >> 32); the 16-bit
- * draw for key j is half (j & 1) of output word ((j & 7) >> 1).  Key j is kept
- * for row i iff that draw is >= T, with T = floor(rate * 65536); kept entries
- * are scaled by 65536 / (65536 - T), the inverse of the exact keep probability.
+ * (i, j >> 4, bh, offset) and the key (seed & 0xffffffff, seed >> 32); the 8-bit
+ * draw for key j is byte (j & 3) of output word ((j & 15) >> 2), so one call
+ * serves 16 keys.  Key j is kept for row i iff that draw is >= T, with
+ * T = floor(rate * 256); kept entries are scaled by 256 / (256 - T), the
+ * inverse of the exact keep probability (the rate takes steps of 1/256).
  *
  * Attention with dropout (the mask applied to the normalised probabilities,
  * after the causal mask and the softmax; the log-sum-exp is the one without
  * dropout):
  *   P_ij  = softmax_j(scale * Q_i . K_j)       (as in ref_attn.c)
- *   Z_ij  = keep_ij * 65536 / (65536 - T)
+ *   Z_ij  = keep_ij * 256 / (256 - T)
  *   O_i   = sum_j P_ij Z_ij V_j,   LSE_i = m_i + ln l_i
  * Backward (chain rule; the softmax Jacobian acts on dP = Z o (dO V^T)):
  *   dP_ij = Z_ij (dO_i . V_j),   D_i = sum_j P_ij dP_ij,   dS_ij = P_ij (dP_ij - D_i)
@@ -67,14 +68,14 @@ void ref_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t ou
     out[3] = c3;
 }
 
-/* The 16-bit draw of (bh, i, j). */
-static uint32_t draw16(uint64_t seed, uint32_t offset, long bh, long i, long j)
+/* The 8-bit draw of (bh, i, j). */
+static uint32_t draw8(uint64_t seed, uint32_t offset, long bh, long i, long j)
 {
-    const uint32_t ctr[4] = {(uint32_t)i, (uint32_t)(j >> 3), (uint32_t)bh, offset};
+    const uint32_t ctr[4] = {(uint32_t)i, (uint32_t)(j >> 4), (uint32_t)bh, offset};
     const uint32_t key[2] = {(uint32_t)(seed & 0xffffffffu), (uint32_t)(seed >> 32)};
     uint32_t w[4];
     ref_philox4x32_10(ctr, key, w);
-    return (w[(j & 7) >> 1] >> (16 * (j & 1))) & 0xffffu;
+    return (w[(j & 15) >> 2] >> (8 * (j & 3))) & 0xffu;
 }
 
 /* keep[bh, i, j] in {0, 1} for every head, row and key. */
@@ -83,7 +84,7 @@ void ref_dropout_mask(long BH, long N, uint64_t seed, uint32_t offset, uint32_t 
     for (long bh = 0; bh < BH; ++bh)
         for (long i = 0; i < N; ++i)
             for (long j = 0; j < N; ++j)
-                keep[(bh * N + i) * N + j] = draw16(seed, offset, bh, i, j) >= T ? 1 : 0;
+                keep[(bh * N + i) * N + j] = draw8(seed, offset, bh, i, j) >= T ? 1 : 0;
 }
 
 /* ------------------------------------------------------ attention + dropout */
@@ -118,7 +119,7 @@ static void prob_row(const double *q, const double *k, long N, long d, double sc
 
 static double zval(uint64_t seed, uint32_t offset, uint32_t T, long bh, long i, long j)
 {
-    return draw16(seed, offset, bh, i, j) >= T ? 65536.0 / (65536.0 - (double)T) : 0.0;
+    return draw8(seed, offset, bh, i, j) >= T ? 256.0 / (256.0 - (double)T) : 0.0;
 }
 
 /* bh0: global head index of the first head passed (the mask's counter uses b*H + h), so

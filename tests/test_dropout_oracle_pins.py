@@ -35,22 +35,22 @@ def test_philox_known_answers():
 
 
 def test_mask_follows_the_counter_layout():
-    """keep[bh,i,j] is half (j&1) of word ((j&7)>>1) of Philox((i, j>>3, bh, offset), seed) compared with T."""
+    """keep[bh,i,j] is byte (j&3) of word ((j&15)>>2) of Philox((i, j>>4, bh, offset), seed) compared with T."""
     BH, N, seed, offset, rate = 3, 40, 0x0123456789ABCDEF, 7, 0.3
     keep = oracle.dropout_mask(BH, N, seed, offset, rate)
     T = oracle.dropout_threshold(rate)
     rng = np.random.default_rng(1)
     for _ in range(200):
         bh, i, j = int(rng.integers(BH)), int(rng.integers(N)), int(rng.integers(N))
-        w = oracle.philox4x32_10([i, j >> 3, bh, offset], [seed & 0xFFFFFFFF, seed >> 32])
-        u = (w[(j & 7) >> 1] >> (16 * (j & 1))) & 0xFFFF
+        w = oracle.philox4x32_10([i, j >> 4, bh, offset], [seed & 0xFFFFFFFF, seed >> 32])
+        u = (w[(j & 15) >> 2] >> (8 * (j & 3))) & 0xFF
         assert keep[bh, i, j] == (1 if u >= T else 0)
 
 
 @pytest.mark.parametrize("rate", [0.1, 0.5, 0.9])
 def test_keep_rate(rate):
     keep = oracle.dropout_mask(4, 256, 42, 0, rate)
-    p = 1.0 - oracle.dropout_threshold(rate) / 65536.0
+    p = 1.0 - oracle.dropout_threshold(rate) / 256.0
     n = keep.size
     assert abs(keep.mean() - p) <= 5.0 * math.sqrt(p * (1 - p) / n)
 
@@ -66,8 +66,8 @@ def test_masks_differ_across_offsets_and_seeds():
 
 def test_threshold_definition():
     assert oracle.dropout_threshold(0.0) == 0
-    assert oracle.dropout_threshold(0.5) == 32768
-    assert oracle.dropout_threshold(0.1) == 6553
+    assert oracle.dropout_threshold(0.5) == 128
+    assert oracle.dropout_threshold(0.1) == 25
     with pytest.raises(ValueError):
         oracle.dropout_threshold(1.0)
 
@@ -90,7 +90,7 @@ def numpy_dropout(q, k, v, do, scale, causal, rate, seed, offset):
     """Whole-matrix restatement: O = (P o Z) V and the matrix chain rule, with Z from the mask."""
     B, H, N, d = q.shape
     T = oracle.dropout_threshold(rate)
-    z = oracle.dropout_mask(B * H, N, seed, offset, rate).reshape(B, H, N, N) * (65536.0 / (65536.0 - T))
+    z = oracle.dropout_mask(B * H, N, seed, offset, rate).reshape(B, H, N, N) * (256.0 / (256.0 - T))
     o_plain, lse, p = np_fwd(q, k, v, scale, causal)
     pz = p * z
     o = pz @ v
@@ -147,7 +147,7 @@ def test_causal_row0_closed_form():
     rate, seed, offset = 0.5, 77, 2
     o, _ = oracle.ref_fwd_dropout(q, k, v, 0.5, True, rate, seed, offset)
     keep = oracle.dropout_mask(B * H, N, seed, offset, rate)
-    inv = 65536.0 / (65536.0 - oracle.dropout_threshold(rate))
+    inv = 256.0 / (256.0 - oracle.dropout_threshold(rate))
     for h in range(H):
         assert np.array_equal(o[0, h, 0], keep[h, 0, 0] * inv * v[0, h, 0])
 
