@@ -54,10 +54,17 @@ __device__ __forceinline__ uint32_t dropout_keep16(const DropoutParams &dp, uint
   return bits;
 }
 
-// bf16-pair mask for a packed word whose low half is key 2c and high half key 2c+1.
-__device__ __forceinline__ uint32_t keep_pair_mask(uint64_t keep, int c) {
-  const uint32_t b = static_cast<uint32_t>(keep >> (2 * c)) & 3u;
-  return ((b & 1u) ? 0x0000FFFFu : 0u) | ((b & 2u) ? 0xFFFF0000u : 0u);
+// Mask for a packed bf16 pair whose low half is key 16*jblk + 2t and high half
+// key 16*jblk + 2t + 1 (t = 0..7), straight from that generator call's words w:
+// 0xFFFF in each half whose key is kept.  The pair's two draw bytes are spread
+// into the two 16-bit halves; adding c256 = (256 - T) * 0x00010001 sets bit 8 of
+// a half exactly when its draw is >= T (the sum stays below 512: no carry
+// between the halves).
+__device__ __forceinline__ uint32_t dropout_pair_mask(const uint4 &w, int t, uint32_t c256) {
+  const uint32_t word = (t >> 1) == 0 ? w.x : (t >> 1) == 1 ? w.y : (t >> 1) == 2 ? w.z : w.w;
+  const uint32_t b0 = static_cast<uint32_t>(2 * t) & 3u;
+  const uint32_t h = __byte_perm(word, 0u, b0 | (4u << 4) | ((b0 + 1u) << 8) | (4u << 12));
+  return (((h + c256) >> 8) & 0x00010001u) * 0xFFFFu;
 }
 
 // Bit c of the keep mask, extracted afresh at each use (volatile: the compiler may

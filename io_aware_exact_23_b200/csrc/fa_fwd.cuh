@@ -434,16 +434,11 @@ __global__ void __launch_bounds__(352, 1)
             for (int cc = 0; cc < 64; ++cc)
               if (cc >= nv) s[cc] = __float_as_uint(-INFINITY);
           }
-          // Dropout: keep bit cc for key j*128 + 64h + cc of query row qt*128 + r,
-          // sixteen keys per generator call (the counter's key block).
-          uint64_t keep = ~0ull;
-          if constexpr (DROPOUT) {
-            keep = 0;
-            const uint32_t jb0 = static_cast<uint32_t>(j * 128 + 64 * h) >> 4;
-  #pragma unroll
-            for (int t = 0; t < 4; ++t)
-              keep |= static_cast<uint64_t>(dropout_keep16(p.drop, qt * 128 + r, jb0 + t, bh)) << (16 * t);
-          }
+          // Dropout: keys j*128 + 64h + 16q .. +15 of query row qt*128 + r come from
+          // generator call jb0 + q (the counter's key block), drawn in the
+          // exponential loop below, one call per 16 keys.
+          const uint32_t jb0 = static_cast<uint32_t>(j * 128 + 64 * h) >> 4;
+          const uint32_t c256 = DROPOUT ? (256u - p.drop.T) * 0x00010001u : 0u;
           // Half-row max as a shallow tree (eight independent chains of four).
           float mq[8];
   #pragma unroll
@@ -487,8 +482,12 @@ __global__ void __launch_bounds__(352, 1)
               return;
             }
             uint64_t acc[2] = {0ull, 0ull}, racc[2] = {0ull, 0ull};
+            uint4 wd = make_uint4(0u, 0u, 0u, 0u);
   #pragma unroll
             for (int cc = 0; cc < 32; ++cc) {
+              if constexpr (DROPOUT) {
+                if ((cc & 7) == 0) wd = dropout_words(p.drop, qt * 128 + r, jb0 + (cc >> 3), bh);
+              }
               const uint64_t x2 = ffma2(f2pack(__uint_as_float(s[2 * cc]), __uint_as_float(s[2 * cc + 1])), c2, n2);
               float x0, x1;
               f2unpack(x2, x0, x1);
@@ -497,7 +496,7 @@ __global__ void __launch_bounds__(352, 1)
               const uint32_t w = pack_bf16(a, b);
               // The sums are of P before dropout; the PV product takes the kept entries
               // (the 1/keep-probability scale is applied to O in the epilogue).
-              pk[cc] = DROPOUT ? (w & keep_pair_mask(keep, cc)) : w;
+              pk[cc] = DROPOUT ? (w & dropout_pair_mask(wd, cc & 7, c256)) : w;
               racc[cc & 1] = fadd2(racc[cc & 1], f2pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
             }
             float u0, u1, u2, u3, v0, v1, v2, v3;
