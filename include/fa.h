@@ -145,7 +145,8 @@ int fa_fwd_fp8(const void *q8, const void *k8, const void *v8,
  * (i, j >> 4, bh, offset) and its key (seed & 0xffffffff, seed >> 32); the
  * 8-bit draw of key j is byte (j & 3) of output word ((j & 15) >> 2); key j is
  * kept for row i iff the draw is >= T = floor(rate * 256) (the rate takes steps
- * of 1/256).  Then
+ * of 1/256: a rate below 1/256 drops nothing, 0.1 drops with probability
+ * 25/256).  Then
  *   O_i = sum_j P_ij * keep_ij * 256/(256 - T) * V_j
  * with P = softmax(scale * Q K^T [+ causal mask]); lse is that of P, without
  * dropout.  The mask is never stored: fa_bwd_dropout regenerates it.

@@ -68,6 +68,8 @@ def test_threshold_definition():
     assert oracle.dropout_threshold(0.0) == 0
     assert oracle.dropout_threshold(0.5) == 128
     assert oracle.dropout_threshold(0.1) == 25
+    assert oracle.dropout_threshold(0.003) == 0  # below 1/256: nothing is dropped
+    assert oracle.dropout_threshold(255.0 / 256.0) == 255
     with pytest.raises(ValueError):
         oracle.dropout_threshold(1.0)
 
