@@ -98,7 +98,7 @@ struct BwdCfg {
   static constexpr int kOffDv = kOffL + 512 * kQStages;       // [kQStages][128] fp32
   static constexpr int kOffBar = kOffDv + 512 * kQStages;
   // then the TMEM address slot, the abort flag and the two-slot unit ring
-  static constexpr int kNumBars = 2 * kQStages + 14;
+  static constexpr int kNumBars = 3 * kQStages + 14;
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static constexpr uint32_t kColS = 0, kColdP = 128, kColdK = 256, kColdV = 256 + D;
@@ -253,13 +253,20 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
   constexpr int S = C::kQStages;  // query tile t sits in stage t % S
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
   uint64_t *bar_kv = bars + 0;
-  uint64_t *bar_qdo_full = bars + 1;       // [S]
-  uint64_t *bar_qdo_empty = bars + 1 + S;  // [S] drain-warp layout: the stage is free again
+  // At d = 64 a stage's loads land on two barriers: Q_i and LSE_i on q_full, dO_i
+  // and D_i on do_full, so that S^T(i) (and P) need not wait for the dO half
+  // (1.03-1.07x there).  At d = 128 the split measured slower (0.97-0.99x: S^T(i)
+  // waits for the issuer's turn behind tile i-1, not for the load) and all four
+  // loads land on q_full.
+  constexpr bool kSplitStage = (D == 64);
+  uint64_t *bar_q_full = bars + 1;             // [S]
+  uint64_t *bar_do_full = bars + 1 + S;        // [S], d = 64
+  uint64_t *bar_qdo_empty = bars + 1 + 2 * S;  // [S] drain-warp layout: the stage is free again
   // [S] compute-drain layout: every compute thread staged its dQ part; without
   // dQ, the issuer's commit after dK(t).  (A per-stage barrier: a wait on it
   // cannot fall two phases behind, which one on dkq_done could across units.)
   uint64_t *bar_staged = bar_qdo_empty;
-  uint64_t *bar_s_full = bars + 1 + 2 * S;
+  uint64_t *bar_s_full = bars + 1 + 3 * S;
   uint64_t *bar_dp_full = bar_s_full + 1;
   uint64_t *bar_p_full = bar_s_full + 2;
   uint64_t *bar_ds_full = bar_s_full + 3;
@@ -270,7 +277,7 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
   uint64_t *bar_unit_full = bar_s_full + 8;   // [2] unit ring: the producer wrote the slot
   uint64_t *bar_unit_empty = bar_s_full + 10; // [2] unit ring: every consumer warp read it
   uint64_t *bar_kv_free = bar_s_full + 12;    // a unit's last MMA completed: K_j, V_j are dead
-  static_assert(1 + 2 * S + 13 == C::kNumBars, "barrier count");
+  static_assert(1 + 3 * S + 13 == C::kNumBars, "barrier count");
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   volatile int *unit_ring = reinterpret_cast<volatile int *>(tmem_slot + 2);  // [2]
@@ -291,17 +298,25 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
 
   const WaitCtx ctx{p.status, abort_flag, kKernelBwd, p.seq};
 
-  // Query tile i of head bh into stage t % S: Q, dO, LSE*log2(e), D.
+  // Query tile i of head bh into stage t % S: Q and LSE*log2(e) on q_full; dO and
+  // D on do_full (d = 64) or on q_full as well (d = 128).
   auto load_tile = [&](int t, int bh, int i) {
     const int s = t % S;
-    mbar_arrive_expect_tx(&bar_qdo_full[s], 2 * C::kTile + 1024);
+    uint64_t *bq = &bar_q_full[s];
+    uint64_t *bd = kSplitStage ? &bar_do_full[s] : bq;
+    if constexpr (kSplitStage) {
+      mbar_arrive_expect_tx(bq, C::kTile + 512);
+      mbar_arrive_expect_tx(bd, C::kTile + 512);
+    } else {
+      mbar_arrive_expect_tx(bq, 2 * C::kTile + 1024);
+    }
     for (int b = 0; b < C::kBoxes; ++b) {
-      tma_load_3d(&tmQ, &bar_qdo_full[s], sQ + s * C::kTile + b * 16384, b * 64, i * 128, bh);
-      tma_load_3d(&tmdO, &bar_qdo_full[s], sdO + s * C::kTile + b * 16384, b * 64, i * 128, bh);
+      tma_load_3d(&tmQ, bq, sQ + s * C::kTile + b * 16384, b * 64, i * 128, bh);
+      tma_load_3d(&tmdO, bd, sdO + s * C::kTile + b * 16384, b * 64, i * 128, bh);
     }
     const size_t soff = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(i) * 128;
-    bulk_load_1d(sL + s * 128, p.ws_lse2 + soff, 512, &bar_qdo_full[s]);
-    bulk_load_1d(sDv + s * 128, p.ws_D + soff, 512, &bar_qdo_full[s]);
+    bulk_load_1d(sL + s * 128, p.ws_lse2 + soff, 512, bq);
+    bulk_load_1d(sDv + s * 128, p.ws_D + soff, 512, bd);
   };
   // Key tile j of head bh: K_j, V_j.
   auto load_kv = [&](int bh, int j) {
@@ -320,7 +335,8 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
     if ((smem_u32(smem) & 1023u) != 0) record_failure(ctx, kStatusInternal, 0);
     mbar_init(bar_kv, 1);
     for (int s = 0; s < S; ++s) {
-      mbar_init(&bar_qdo_full[s], 1);
+      mbar_init(&bar_q_full[s], 1);
+      mbar_init(&bar_do_full[s], 1);
       // bar_staged in the compute-drain layout: 256 stagers, or the issuer's commit
       mbar_init(&bar_qdo_empty[s], R::kComputeDrain ? (NO_DQ ? 1 : 256) : 1);
     }
@@ -380,14 +396,19 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
       int n_loaded = 0;     // query tiles whose loads were issued
       int n_kv = 0;         // K/V loads issued
       int stage_row[S] = {}, stage_bh[S] = {};  // the tile each stage holds
-      // Compute-drain layout: query tile t's stage is reloaded (for tile t + S)
-      // once the tile is done with -- after the issuer's commit behind dK(t)
+      // Compute-drain layout: query tile tt's stage is reloaded (for tile tt + S)
+      // once the tile is done with -- after the issuer's commit behind dK(tt)
       // without the dQ product; else once every compute thread has staged its
-      // part of dQ(t) there and this thread has reduce-added the staged tile into
-      // the accumulator (and TMA has read it).
-      auto free_stage = [&](int tt) -> bool {
+      // part of dQ(tt) there and this thread has reduce-added the staged tile into
+      // the accumulator and TMA has read it.  (Reloading Q as soon as the Q
+      // buffer's half had been read measured no faster: at d = 128, S^T(tt + S)
+      // waits for the issuer's turn behind tile tt + S - 1, not for the stage.)
+      // reload = false: the last S tiles, with no load behind them.
+      auto free_stage = [&](int tt, bool reload, int bh, int i) -> bool {
         const int st = tt % S;
+        if (tt < 256) FA_TRACE(3000 + tt * 3 + 0);
         if (!mbar_wait(ctx, &bar_staged[st], (tt / S) & 1, kBTagStage)) return false;
+        if (tt < 256) FA_TRACE(3000 + tt * 3 + 1);
         if constexpr (!NO_DQ) {
           for (int half = 0; half < 2; ++half)
             for (int b = 0; b < D / 64; ++b)
@@ -395,7 +416,9 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
                                 half * (D / 2) + 32 * b, stage_row[st], stage_bh[st]);
           bulk_commit();
           bulk_wait_read<0>();
+          if (tt < 256) FA_TRACE(3000 + tt * 3 + 2);
         }
+        if (reload) load_tile(tt + S, bh, i);
         return true;
       };
       int unit = static_cast<int>(blockIdx.x) < n_units ? static_cast<int>(blockIdx.x) : -1;
@@ -414,11 +437,15 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
             n_loaded = n_kv = 1;
           } else {
             if constexpr (R::kComputeDrain) {
-              if (t >= S && !(ok = free_stage(t - S))) break;
-            } else if (n > 0 && !(ok = mbar_wait(ctx, &bar_qdo_empty[s], (n - 1) & 1, kBTagQdoEmpty))) {
-              break;
+              if (t >= S) {
+                if (!(ok = free_stage(t - S, true, bh, i0 + it))) break;
+              } else {
+                load_tile(t, bh, i0 + it);
+              }
+            } else {
+              if (n > 0 && !(ok = mbar_wait(ctx, &bar_qdo_empty[s], (n - 1) & 1, kBTagQdoEmpty))) break;
+              load_tile(t, bh, i0 + it);
             }
-            load_tile(t, bh, i0 + it);
             ++n_loaded;
             if (it == 0) {
               // K_j, V_j of this unit, once every MMA of the previous one has
@@ -445,7 +472,7 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
       if constexpr (R::kComputeDrain && !NO_DQ) {
         // The last S tiles have no load behind them: reduce-add their staged dQ
         // here.  (Without the dQ product there is nothing to wait for.)
-        for (int tt = t >= S ? t - S : 0; tt < t && ok; ++tt) ok = free_stage(tt);
+        for (int tt = t >= S ? t - S : 0; tt < t && ok; ++tt) ok = free_stage(tt, false, 0, 0);
         bulk_wait<0>();  // every reduction has landed before the CTA exits
       }
       // The last loads have landed before the CTA can exit (immediate unless a
@@ -453,7 +480,8 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
       if (n_kv > 0) mbar_drain(bar_kv, (n_kv - 1) & 1);
       for (int s = 0; s < S && s < n_loaded; ++s) {
         const int last = s + ((n_loaded - 1 - s) / S) * S;
-        mbar_drain(&bar_qdo_full[s], (last / S) & 1);
+        mbar_drain(&bar_q_full[s], (last / S) & 1);
+        if (kSplitStage) mbar_drain(&bar_do_full[s], (last / S) & 1);
       }
     }
     __syncwarp();
@@ -523,9 +551,9 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
         mma_commit_w(bar_dkq_done);
         if (lane == 0) FA_TRACE(16 + t * 8 + 3);
       };
-      auto wait_stage = [&](int t) {
-        return wait(&bar_qdo_full[t % S], (t / S) & 1, kBTagQdoFull);
-      };
+      // Tile t's Q and LSE (for S^T, dK) and its dO and D (for dP^T, dV).
+      auto wait_q = [&](int t) { return wait(&bar_q_full[t % S], (t / S) & 1, kBTagQdoFull); };
+      auto wait_do = [&](int t) { return !kSplitStage || wait(&bar_do_full[t % S], (t / S) & 1, kBTagQdoFull); };
       // S^T(i+1) overwrites P^T(i), which dV(i) reads, and dP^T(i+1) the dP^T(i)
       // the compute warps have turned into dS(i): neither waits for an MMA to
       // complete, since one lane issues them all and the pipe runs them in order.
@@ -544,9 +572,11 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
           // next tile's S^T goes in ahead of dK(i) (and dQ(i), which has columns of
           // its own at d = 64), so the compute warps start tile i+1 while those run.
           // Without dQ, dK(i)'s commit closes the tile and frees its stage.
-          if (!(ok = wait_stage(t0))) break;
+          if (!(ok = wait_q(t0))) break;
           tc_fence_after();
           issue_sT(t0);
+          if (!(ok = wait_do(t0))) break;
+          tc_fence_after();
           issue_dPT(t0);
           for (int it = 0; it < n_it && ok; ++it) {
             t = t0 + it;
@@ -554,7 +584,7 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
             tc_fence_after();
             issue_dV(t, it > 0);
             if (it + 1 < n_it) {
-              if (!(ok = wait_stage(t + 1))) break;
+              if (!(ok = wait_q(t + 1))) break;
               tc_fence_after();
               issue_sT(t + 1);
             }
@@ -571,20 +601,23 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
               }
               issue_dQ(t);
             }
-            if (it + 1 < n_it) issue_dPT(t + 1);
+            if (it + 1 < n_it) {
+              if (!(ok = wait_do(t + 1))) break;
+              tc_fence_after();
+              issue_dPT(t + 1);
+            }
           }
         } else {
           // Order S^T(i) dP^T(i) dV(i) dK(i) dQ(i).  dQ(i) accumulates in dP^T's
           // columns, so dP^T(i+1) also waits for the drain to have read dQ(i).
           for (int it = 0; it < n_it && ok; ++it) {
             t = t0 + it;
-            if (!(ok = wait_stage(t))) break;
+            if (!(ok = wait_q(t))) break;
             tc_fence_after();
             issue_sT(t);
-            if (t > 0) {
-              if (!(ok = wait(bar_dq_empty, (t - 1) & 1, kBTagDqEmpty))) break;
-              tc_fence_after();
-            }
+            if (t > 0 && !(ok = wait(bar_dq_empty, (t - 1) & 1, kBTagDqEmpty))) break;
+            if (!(ok = wait_do(t))) break;
+            tc_fence_after();
             issue_dPT(t);
             if (!(ok = wait(bar_p_full, t & 1, kBTagPFull))) break;
             tc_fence_after();
@@ -635,7 +668,7 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
         const int t = t0 + it;
         const int s = t % S, n = t / S;
         ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_s_full, t & 1, kBTagSFull) &&
-                                         mbar_wait(ctx, &bar_qdo_full[s], n & 1, kBTagQdoFull));
+                                         mbar_wait(ctx, &bar_q_full[s], n & 1, kBTagQdoFull));
         if (!ok) break;
         tc_fence_after();
         if (threadIdx.x == 0) FA_TRACE(16 + t * 8 + 4);
@@ -692,7 +725,10 @@ __global__ void __launch_bounds__(BwdRoles<D, NO_DQ>::kThreads, 1)
         mbar_arrive(bar_p_full);
         if (threadIdx.x == 0) FA_TRACE(16 + t * 8 + 5);
 
-        ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dp_full, t & 1, kBTagDpFull));
+        // dP^T, and D (it came with dO: the issuer waited for both before dP^T, but
+        // the data's visibility to these threads comes with their own wait).
+        ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dp_full, t & 1, kBTagDpFull) &&
+                                         (!kSplitStage || mbar_wait(ctx, &bar_do_full[s], n & 1, kBTagQdoFull)));
         // The previous tile's dK / dQ MMAs read dS from smem: wait until they are done.
         if (ok && t > 0) ok = __all_sync(0xffffffffu, mbar_wait(ctx, bar_dkq_done, (t - 1) & 1, kBTagDkqDone));
         if (!ok) break;

@@ -6,7 +6,9 @@ j, with its query tiles); its tiles are numbered across units (t), and every
 per-tile barrier phase and stage follows t.  Roles, as in the kernel:
   * producer: hands each unit to the other roles through a two-slot ring (the
     kernel fetches the next unit from a counter); per tile t, Q_t, dO_t, LSE_t,
-    D_t into stage t % S (S = 3 stages at d = 64, 2 at d = 128).  With drain
+    D_t into stage t % S (S = 3 stages at d = 64, 2 at d = 128); at d = 64 Q and
+    LSE land on one barrier, dO and D on another, which S^T and dP^T wait for
+    separately.  With drain
     warps (d = 64) it reloads a stage after its "empty" barrier; in the
     compute-drain layout (d = 128, and every no-dQ instantiation) it frees tile
     t - S's stage itself just before reloading it: it waits for the compute warps'
@@ -66,7 +68,10 @@ def bwd_model(units, d: int, seed: int, dropout: bool = False, skip: str = "", n
     compute_drain = d == 128 or no_dq  # the kernel's BwdRoles::kComputeDrain
     S = 3 if d == 64 else 2  # the kernel's BwdCfg::kQStages: tile t sits in stage t % S
     bar_kv = Bar("kv", 2)
-    qdo_full = [Bar(f"qdo_full{s}", 4) for s in range(S)]  # Q, dO, LSE, D
+    # d = 64: Q, LSE on q_full and dO, D on do_full; d = 128: all four on q_full.
+    split = d == 64
+    q_full = [Bar(f"q_full{s}", 2 if split else 4) for s in range(S)]
+    do_full = [Bar(f"do_full{s}", 2) for s in range(S)] if split else q_full
     qdo_empty = [Bar(f"qdo_empty{s}", 1) for s in range(S)]
     # compute-drain layout: every compute warp staged its dQ part; without dQ, the
     # issuer's commit after dK(t) (a per-stage barrier: a wait on it cannot fall two
@@ -89,16 +94,35 @@ def bwd_model(units, d: int, seed: int, dropout: bool = False, skip: str = "", n
         M.read(("ring", u & 1), u if u < n_units else None)
         unit_empty[u & 1].arrive()
 
-    def free_stage(t):
-        """Compute-drain layout: the producer frees tile t's stage."""
+    def load_q(t):
+        M.load(("Q", t % S), ("Q", t), q_full[t % S])
+        M.load(("L", t % S), ("L", t), q_full[t % S])
+
+    def load_do(t):
+        M.load(("dO", t % S), ("dO", t), do_full[t % S])
+        M.load(("Dv", t % S), ("Dv", t), do_full[t % S])
+
+    def free_stage(t, reload=None):
+        """Compute-drain layout: the producer frees tile t's stage (and loads tile
+        `reload` into it) once the reduce-add has read the staged dQ."""
         st = t % S
         if no_dq:
             yield lambda: staged[st].ready(t // S)
+            if reload is not None:
+                load_q(reload)
+                load_do(reload)
             return
         if skip != "staged_wait":
             yield lambda: staged[st].ready(t // S)
+        if skip == "early_q_reload" and reload is not None:
+            load_q(reload)  # wrong: before the reduce-add has read the Q buffer
         M.read(("Q", st), ("dQ staged", t))  # the reduce-add's read (waited for)
+        yield lambda: True
         M.read(("dO", st), ("dQ staged", t))
+        if reload is not None:
+            if skip != "early_q_reload":
+                load_q(reload)
+            load_do(reload)
 
     def producer():
         yield lambda: True
@@ -112,13 +136,13 @@ def bwd_model(units, d: int, seed: int, dropout: bool = False, skip: str = "", n
             for it in range(units[u]):
                 t = first[u] + it
                 s, n = t % S, t // S
-                if compute_drain:
-                    if t >= S:
-                        yield from free_stage(t - S)
-                elif n > 0:
-                    yield lambda s=s, n=n: qdo_empty[s].ready(n - 1)
-                for nm in ("Q", "dO", "L", "Dv"):
-                    M.load((nm, s), (nm, t), qdo_full[s])
+                if compute_drain and t >= S:
+                    yield from free_stage(t - S, reload=t)
+                else:
+                    if not compute_drain and n > 0:
+                        yield lambda s=s, n=n: qdo_empty[s].ready(n - 1)
+                    load_q(t)
+                    load_do(t)
                 if it == 0:
                     # K_j, V_j of this unit: after every MMA of the previous one (a
                     # per-unit barrier: a wait on dkq_done(t-1) could pass early
@@ -134,8 +158,11 @@ def bwd_model(units, d: int, seed: int, dropout: bool = False, skip: str = "", n
                     yield from free_stage(t)
 
     def issuer():
-        def stage_ready(t):
-            return lambda: qdo_full[t % S].ready(t // S)
+        def q_ready(t):
+            return lambda: q_full[t % S].ready(t // S)
+
+        def do_ready(t):
+            return lambda: do_full[t % S].ready(t // S)
 
         for u in range(n_units + 1):
             yield from get_unit(u)
@@ -179,28 +206,32 @@ def bwd_model(units, d: int, seed: int, dropout: bool = False, skip: str = "", n
             yield lambda: bar_kv.ready(u)
             if no_dq:
                 # S^T(first) dP^T(first) | dV(t) S^T(t+1) [dS] dK(t) dP^T(t+1) | ... at both d
-                yield stage_ready(t0)
+                yield q_ready(t0)
                 sT(t0)
+                yield do_ready(t0)
                 dPT(t0)
                 for it in range(n_it):
                     t = t0 + it
                     yield lambda t=t: p_full.ready(t)
                     dV(t)
                     if it + 1 < n_it:
-                        yield stage_ready(t + 1)
+                        yield q_ready(t + 1)
                         sT(t + 1)
                     if skip != "ds_wait":
                         yield lambda t=t: ds_full.ready(t)
                     dK(t)
                     if it + 1 < n_it:
+                        yield do_ready(t + 1)
                         dPT(t + 1)
             elif d == 128:
                 for it in range(n_it):
                     t = t0 + it
-                    yield stage_ready(t)
+                    yield q_ready(t)
                     sT(t)
                     if t > 0:
                         yield lambda t=t: dq_empty.ready(t - 1)
+                    if skip != "do_wait":
+                        yield do_ready(t)
                     dPT(t)
                     yield lambda t=t: p_full.ready(t)
                     dV(t)
@@ -209,15 +240,16 @@ def bwd_model(units, d: int, seed: int, dropout: bool = False, skip: str = "", n
                     dK(t)
                     dQ(t)
             else:
-                yield stage_ready(t0)
+                yield q_ready(t0)
                 sT(t0)
+                yield do_ready(t0)
                 dPT(t0)
                 for it in range(n_it):
                     t = t0 + it
                     yield lambda t=t: p_full.ready(t)
                     dV(t)
                     if it + 1 < n_it:
-                        yield stage_ready(t + 1)
+                        yield q_ready(t + 1)
                         sT(t + 1)
                     yield lambda t=t: ds_full.ready(t)
                     dK(t)
@@ -225,6 +257,7 @@ def bwd_model(units, d: int, seed: int, dropout: bool = False, skip: str = "", n
                         yield lambda t=t: dq_empty.ready(t - 1)
                     dQ(t)
                     if it + 1 < n_it:
+                        yield do_ready(t + 1)
                         dPT(t + 1)
             M.commit(0, kv_free)
 
@@ -237,7 +270,7 @@ def bwd_model(units, d: int, seed: int, dropout: bool = False, skip: str = "", n
             for it in range(n_it):
                 t = t0 + it
                 s, n = t % S, t // S
-                yield lambda t=t, s=s, n=n: s_full.ready(t) and qdo_full[s].ready(n)
+                yield lambda t=t, s=s, n=n: s_full.ready(t) and q_full[s].ready(n)
                 if dropout:
                     if t > 0 and skip != "draws_wait":
                         yield lambda t=t: dkq_done.ready(t - 1)
@@ -250,6 +283,7 @@ def bwd_model(units, d: int, seed: int, dropout: bool = False, skip: str = "", n
                 yield lambda t=t: dp_full.ready(t)
                 if t > 0:  # implied by dp_full(t): dP^T(t) is issued after dQ(t-1)
                     yield lambda t=t: dkq_done.ready(t - 1)
+                yield lambda s=s, n=n: do_full[s].ready(n)
                 M.read(("dPT", w, q), ("dP", t))
                 M.read(("Dv", s), ("Dv", t))
                 M.write(("dS", w, q), ("dS", t))
@@ -362,11 +396,14 @@ def test_no_dq_model_detects_a_missing_wait():
     assert failures > 0
 
 
-@pytest.mark.parametrize("skip", ["staged_wait", "drain_wait"])
+@pytest.mark.parametrize("skip", ["staged_wait", "drain_wait", "early_q_reload"])
 def test_compute_drain_model_detects_a_missing_wait(skip):
     """Not vacuous for the compute-drain layout: a producer that reduce-adds and
-    reloads a stage without waiting for every warp's staged dQ, or compute warps
-    that read dQ before dK / dQ completed, fail the model."""
+    reloads a stage without waiting for every warp's staged dQ, or that reloads
+    Q before the reduce-add has read it, or compute warps that read dQ before
+    dK / dQ completed, fail the model.  (The issuer's wait for dO(t) before
+    dP^T(t) has no such control here: dO loads together with Q, which S^T(t)
+    waited for, and dP^T(t) also waits for the drain of dQ(t-1).)"""
     failures = 0
     for seed in range(40):
         try:
