@@ -19,7 +19,7 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("B,H,N,rate,seed,offset", [
     (1, 3, 200, 0.1, 0, 0), (2, 2, 130, 0.5, 0xFEDCBA9876543210, 7), (1, 1, 17, 0.9, 12345, 1 << 31),
-    (1, 2, 64, 0.0, 3, 3)])
+    (1, 2, 64, 0.0, 3, 3), (1, 1, 33, 0.003, 5, 0)])
 def test_mask_is_bit_exact(B, H, N, rate, seed, offset):
     mask = torch.full((B, H, N, N), 7, dtype=torch.uint8, device="cuda")
     fa.fa_dropout_mask(B, H, N, rate, seed, offset, mask)
@@ -66,11 +66,13 @@ def test_dropout_matches_oracle(w, rate):
     check_grads({"dq": to64(dq), "dk": to64(dk), "dv": to64(dv)}, {"dq": rq, "dk": rk, "dv": rv}, w.name)
 
 
-@pytest.mark.parametrize("d,causal", [(64, False), (128, True)])
-def test_rate_zero_is_the_plain_kernel(d, causal):
+@pytest.mark.parametrize("d,causal,rate", [(64, False, 0.0), (128, True, 0.0), (128, False, 0.003)])
+def test_rate_zero_is_the_plain_kernel(d, causal, rate):
+    """Rate 0, or any rate below 1/256 (the rate's step: T = 0, every key kept,
+    scale 1), reproduces the dropout-free kernels."""
     w = Workload("drop0", 2, 3, 700, d, causal, seed=8)
     t = make_inputs(w, device="cuda")
-    o, lse, _, dq, dk, dv = run_dropout(t, w, 0.0, 1, 0, residual=False)
+    o, lse, _, dq, dk, dv = run_dropout(t, w, rate, 1, 0, residual=False)
     o2 = torch.empty_like(o)
     lse2 = torch.empty_like(lse)
     fa.fa_fwd(t["q"], t["k"], t["v"], o2, lse2, w.scale, causal)
