@@ -24,7 +24,7 @@
 // over S columns [64h, 64h+32) -- inside the half its warp has already read --
 // and is the A operand of the PV MMA straight from TMEM.  The next S of a tile
 // overwrites those columns; its issuer puts it in the pipe right behind that
-// tile's PV (one issuing thread: the MMAs execute in order), without waiting.
+// tile's PV (one issuing lane: the MMAs execute in order), without waiting.
 //
 // Online softmax, in the log2 domain with c = scale*log2(e):
 //   m' = max(m, c*rowmax(S));  P = 2^(c*S - m');  l = 2^(m-m') l + rowsum(P);
@@ -298,8 +298,8 @@ __global__ void __launch_bounds__(352, 1)
     // ------------------------------------------------------------ MMA issuers
     // The whole warp runs the issue loop (waits, unit decode, descriptors), so
     // that every value it computes is warp-uniform; one elected lane issues each
-    // MMA and commit.  Run from a single lane, the same loop took about 100 SM
-    // cycles per MMA while the softmax warps kept the sub-partition busy.
+    // MMA and commit.  (Run from a single lane, the loop took about 100 SM cycles
+    // per MMA while the softmax warps kept the sub-partition busy; 60-70 this way.)
     const int k = __shfl_sync(0xffffffffu, warp, 0) - C::kIssuerWarp;  // query tile owned by this issuer
     const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
     if (__all_sync(0xffffffffu, *abort_flag == 0)) {
