@@ -783,8 +783,27 @@ def main():
         if fa.fa_device_status() != 0:
             raise SystemExit("bench.py: device status error in the e2e leg")
         e2e_ms = reduce_max([e0.elapsed_time(e1) / E], dist, dev)[0]
+        # The host link's floor for the same bytes: the same copies, both directions
+        # at once on their two streams, with no kernels between them.
+        torch.cuda.synchronize()
+        c0, c1 = mk(), mk()
+        c0.record(s_in)
+        s_out.wait_stream(s_in)
+        for st in range(E):
+            D, Hh = dev_sets[st % 2], host_out[st % 2]
+            with torch.cuda.stream(s_in):
+                for nm in names_in:
+                    D[nm].copy_(pin[nm], non_blocking=True)
+            with torch.cuda.stream(s_out):
+                for nm in names_out:
+                    Hh[nm].copy_(D[nm], non_blocking=True)
+        s_in.wait_stream(s_out)
+        c1.record(s_in)
+        torch.cuda.synchronize()
+        copy_ms = reduce_max([c0.elapsed_time(c1) / E], dist, dev)[0]
         e2e = {"value": world * (w.fwd_flops() + w.bwd_flops()) / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": E,
+               "copies_alone_ms_per_step": copy_ms, "copy_floor_frac": copy_ms / e2e_ms,
                "path": "pinned host -> device copies, fa_fwd + fa_bwd through the C ABI, outputs -> pinned host; "
                        "two buffer sets, copy-in / compute / copy-out streams overlapped across steps"}
 
