@@ -552,20 +552,18 @@ __global__ void __launch_bounds__(352, 1)
       }
       if (!ok) break;
       // -------------------------------------------------------- epilogue
-      // Once both tiles' last PV of the unit has completed, O_k is final.  Each
-      // warp turns its 32 rows x D/2 columns of O_k (and of the rounding
+      // Once tile k's last PV of the unit has completed, O_k is final (tile 0's
+      // epilogue runs while tile 1's last PV does).  Each warp turns its 32 rows x D/2 columns of O_k (and of the rounding
       // residual) into bf16 32 columns at a time, stages them in its own 2 KB
       // (16-byte chunks XOR-swizzled by row pair, so that the row-wise writes and
       // the chunk-wise read-back are free of bank conflicts) and writes them out
       // with 16-byte stores covering whole 64-byte row segments.  The staging is
       // its own, so the next unit's loads and first S MMAs run meanwhile, and
       // nothing waits for the stores.
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait(ctx, &bar_pv_done[0], (cs[0] + n_k[0] - 1) & 1, kTagPvDone) &&
-                          mbar_wait(ctx, &bar_pv_done[1], (cs[1] + n_k[1] - 1) & 1, kTagPvDone));
-      if (!ok) break;
-      tc_fence_after();
       for (int k = 0; k < 2 && ok; ++k) {
+        ok = __all_sync(0xffffffffu, mbar_wait(ctx, &bar_pv_done[k], (cs[k] + n_k[k] - 1) & 1, kTagPvDone));
+        if (!ok) break;
+        tc_fence_after();
         const int qt = 2 * u + k;
         // Whole-row sums from the two column halves.
         float *ls = reinterpret_cast<float *>(smem + C::kLOff) + k * 512;  // [h][2][128]

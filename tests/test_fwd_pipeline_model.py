@@ -177,8 +177,9 @@ def fwd_model(units, stages: int, seed: int, pv_without_p_wait: bool = False, sk
                     M.write(("S", k, h, rq), ("P", u, j))
                     p_full[k].arrive()
             last = [cs[u][k] + n_k[k] - 1 for k in range(2)]
-            yield lambda last=last: pv_done[0].ready(last[0]) and pv_done[1].ready(last[1])
-            for k in range(2):
+            for k in range(2):  # tile 0's epilogue runs while tile 1's last PV does
+                if not (skip == "epi_wait" and k == 1):
+                    yield lambda k=k, t=last[k]: pv_done[k].ready(t)
                 M.write(("ls", k, h, rq), ("sum", u))
                 bar_l[k][rq].arrive()
                 yield lambda k=k, u=u: bar_l[k][rq].ready(u)
@@ -238,6 +239,18 @@ def test_persistent_model_detects_an_early_q_reload():
     for seed in range(60):
         try:
             fwd_model([(3, 4), (2, 2), (3, 4)], 4, seed, skip="q_free")
+        except AssertionError:
+            failures += 1
+    assert failures > 0
+
+
+def test_model_detects_a_missing_epilogue_wait():
+    """Not vacuous: reading O_1 in the epilogue without waiting for its own last PV
+    (only for tile 0's) fails the model."""
+    failures = 0
+    for seed in range(60):
+        try:
+            fwd_model([(3, 4), (2, 2)], 4, seed, skip="epi_wait")
         except AssertionError:
             failures += 1
     assert failures > 0
