@@ -553,8 +553,9 @@ __global__ void __launch_bounds__(352, 1)
       if (!ok) break;
       // -------------------------------------------------------- epilogue
       // Once tile k's last PV of the unit has completed, O_k is final (tile 0's
-      // epilogue runs while tile 1's last PV does).  Each warp turns its 32 rows x D/2 columns of O_k (and of the rounding
-      // residual) into bf16 32 columns at a time, stages them in its own 2 KB
+      // epilogue runs while tile 1's last PV does).  Each warp turns its 32 rows
+      // x D/2 columns of O_k (and of the rounding residual) into bf16 32 columns
+      // at a time, stages them in its own 2 KB
       // (16-byte chunks XOR-swizzled by row pair, so that the row-wise writes and
       // the chunk-wise read-back are free of bank conflicts) and writes them out
       // with 16-byte stores covering whole 64-byte row segments.  The staging is
